@@ -1,0 +1,128 @@
+"""Seeded synthetic inputs shared by the CUDA path's tests/bench and the oracle.
+
+This module draws random numbers and lays out shapes; it holds none of the
+method's arithmetic (no norm, no rotation, no softmax, no positions).  Both
+sides receive the same bf16 bit patterns.
+
+Recipe: every tensor is drawn from a CPU ``torch.Generator`` seeded with
+``seed * 16 + stream`` (streams: q=0, k=1, v=2, cache pre-fill=3, gains=4),
+as float32 N(0, 1) and rounded to bf16 by torch (round-to-nearest-even).
+Gains are ``1 + 0.1 * N(0, 1)`` in float32.  Unit-scale N(0,1) activations
+stand in for the projections of a trained Wan-style DiT layer (no weights
+are available); the shapes follow the workloads named below.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+import torch
+
+STREAM_Q, STREAM_K, STREAM_V, STREAM_CACHE, STREAM_GAMMA = 0, 1, 2, 3, 4
+
+
+@dataclass(frozen=True)
+class Workload:
+    """Shape of one wave round.
+
+    L: tokens per chunk (= F * gh * gw); n_wave: chunks in the wave (denoising
+    chunks + 1 refresh chunk); n_hist: history chunks in the ring; H, D: heads
+    and head_dim; F, gh, gw: latent frames per chunk and the patch grid.
+    """
+    name: str
+    H: int
+    D: int
+    F: int
+    gh: int
+    gw: int
+    n_wave: int
+    n_hist: int
+    layers: int = 1
+    rounds: int = 1
+
+    @property
+    def L(self) -> int:
+        return self.F * self.gh * self.gw
+
+    @property
+    def T(self) -> int:
+        return self.n_wave * self.L
+
+    @property
+    def R(self) -> int:
+        return self.n_hist + self.n_wave
+
+
+# The five workloads of the wave-round hot path.
+WORKLOADS = {
+    "tiny": Workload("tiny: 2x64, 3 chunks x 32 tokens (2x4x4), no history",
+                     H=2, D=64, F=2, gh=4, gw=4, n_wave=3, n_hist=0),
+    "wan13b_4step": Workload("wan1.3b 4-step wave: 12x128, 5 chunks x 4680 (3x30x52), history 2",
+                             H=12, D=128, F=3, gh=30, gw=52, n_wave=5, n_hist=2),
+    "wan13b_5step": Workload("wan1.3b 5-step wave: 12x128, 6 chunks x 4680, history 3",
+                             H=12, D=128, F=3, gh=30, gw=52, n_wave=6, n_hist=3),
+    "wan13b_round": Workload("wan1.3b full round: 30 layers of the 4-step wave, 20 rounds",
+                             H=12, D=128, F=3, gh=30, gw=52, n_wave=5, n_hist=2,
+                             layers=30, rounds=20),
+    "wan14b_4step": Workload("wan14b 4-step wave: 40x128, 5 chunks x 4680, history 3",
+                             H=40, D=128, F=3, gh=30, gw=52, n_wave=5, n_hist=3),
+}
+
+
+def _gen(seed: int, stream: int) -> torch.Generator:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed) * 16 + int(stream))
+    return g
+
+
+def bf16_normal(shape, seed: int, stream: int) -> torch.Tensor:
+    """bf16 CPU tensor of N(0,1) draws, rounded from float32."""
+    x = torch.randn(tuple(shape), generator=_gen(seed, stream), dtype=torch.float32)
+    return x.to(torch.bfloat16)
+
+
+def gains(H: int, D: int, seed: int) -> "tuple[torch.Tensor, torch.Tensor]":
+    """(gamma_q, gamma_k) float32 [H, D], each 1 + 0.1*N(0,1)."""
+    g = torch.randn((2, H, D), generator=_gen(seed, STREAM_GAMMA), dtype=torch.float32)
+    return (1.0 + 0.1 * g[0]).contiguous(), (1.0 + 0.1 * g[1]).contiguous()
+
+
+@dataclass
+class WaveInputs:
+    q: torch.Tensor          # bf16 [T, H, D]
+    k: torch.Tensor          # bf16 [T, H, D]
+    v: torch.Tensor          # bf16 [T, H, D]
+    gamma_q: torch.Tensor    # f32 [H, D]
+    gamma_k: torch.Tensor    # f32 [H, D]
+
+
+def wave_inputs(w: Workload, seed: int = 0, salt: int = 0) -> WaveInputs:
+    """q, k, v of one wave round plus the RMSNorm gains.
+
+    ``salt`` gives further independent draws (other layers, other rounds).
+    """
+    s = seed + 1009 * salt
+    shape = (w.T, w.H, w.D)
+    gq, gk = gains(w.H, w.D, seed)
+    return WaveInputs(bf16_normal(shape, s, STREAM_Q), bf16_normal(shape, s, STREAM_K),
+                      bf16_normal(shape, s, STREAM_V), gq, gk)
+
+
+def history_prefill(w: Workload, n_chunks: Optional[int] = None, seed: int = 0,
+                    salt: int = 0) -> "tuple[torch.Tensor, torch.Tensor]":
+    """Clean history K/V [n_chunks, L, H, D] bf16 to seed the ring before round n_hist."""
+    n = w.n_hist if n_chunks is None else n_chunks
+    g = torch.randn((2, n, w.L, w.H, w.D), generator=_gen(seed + 1009 * salt, STREAM_CACHE),
+                    dtype=torch.float32).to(torch.bfloat16)
+    return g[0].contiguous(), g[1].contiguous()
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    """bf16 tensor -> numpy uint16 bit patterns (same memory order)."""
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def from_bits(a: np.ndarray) -> torch.Tensor:
+    """numpy uint16 bit patterns -> bf16 tensor."""
+    return torch.from_numpy(np.ascontiguousarray(a, np.uint16).view(np.int16)).view(torch.bfloat16)

@@ -1,0 +1,265 @@
+/*
+ * wf_oracle.c -- CPU fp64 oracle for the Wave Forcing wave-round hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path links, loads or calls
+ * this file: only the test suite, the smoke check and the CPU-baseline leg of
+ * the benchmark do.  It shares no code, header, table or helper with the CUDA
+ * library; the two meet only through seeded input arrays.
+ *
+ * What it computes (all arithmetic in IEEE double, plain loops, no blocking):
+ *
+ *   wfo_bf16_to_f64 / wfo_f64_to_bf16
+ *       exact widening of bf16 bit patterns, and round-to-nearest-even
+ *       narrowing straight from double (IEEE 754 definition of RNE).
+ *
+ *   wfo_positions
+ *       (t,h,w) of every wave token: wave chunk c of round r is absolute chunk
+ *       g = r + c; token n = c*L + f*gh*gw + y*gw + x has t = g*F + f, h = y,
+ *       w = x.  (The pages fix 3-latent-frame chunks and a 480x832 grid, see
+ *       "Wave Forcing", airadar.tv summary, usage notes on --num-frames; the
+ *       absolute-time reading is ours, parity for it is pinned by closed form.)
+ *
+ *   wfo_append
+ *       per (token, head): per-head RMSNorm of q and k with gain gamma[h,:],
+ *       then 3D RoPE on (t,h,w), then one rounding to bf16; v is copied.
+ *       The pages name no norm or RoPE formula (they are fixed by the problem
+ *       statement of the hot path); the readings are:
+ *         y_d = x_d * gamma_d / sqrt(mean_d x_d^2 + eps)
+ *         channels [0,dt) rotate with t, [dt,dt+dh) with h, [dt+dh,D) with w;
+ *         pair (2i, 2i+1) of an axis block of width da turns by pos*theta^(-2i/da).
+ *
+ *   wfo_chunk_causal_attn_rows
+ *       softmax attention of selected (query row, head) pairs over an explicit
+ *       concatenation of key chunks, each tagged with its absolute chunk id.
+ *       Key j is visible to query n exactly when chunk_id(j) <= chunk_id(n):
+ *       later chunks see earlier (cleaner) chunks and all of their own chunk,
+ *       never a later chunk ("Wave Forcing" abstract: chunk-wise causal
+ *       attention reaching earlier, cleaner chunks before their denoising is
+ *       complete).  s_j = q.k_j / sqrt(D); p = softmax over visible j;
+ *       O = sum_j p_j v_j; lse = m + log(sum_j exp(s_j - m)).
+ *
+ * Parity pins live in tests/test_oracle_pins.py (brute-force dense mask,
+ * library softmax attention on the unmasked special case, closed forms and
+ * invariants).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ---- bf16 <-> double ---------------------------------------------------- */
+
+static double bf16_bits_to_double(uint16_t b)
+{
+    uint32_t u = ((uint32_t)b) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Round-to-nearest, ties-to-even, from double to bf16 (8 significand bits,
+ * 8 exponent bits).  Works on the real value: find the bf16 quantum q of the
+ * binade holding |x|, take rint(x / q) (the C default rounding mode is
+ * nearest-even), multiply back.  The result is a float-representable value,
+ * whose top 16 bits are the bf16 pattern. */
+static uint16_t double_to_bf16_bits(double x)
+{
+    if (isnan(x)) return 0x7FC0u;
+    if (isinf(x)) return x > 0 ? 0x7F80u : 0xFF80u;
+    if (x == 0.0) return signbit(x) ? 0x8000u : 0x0000u;
+    int e2;
+    (void)frexp(fabs(x), &e2);          /* |x| = m * 2^e2, m in [0.5, 1) */
+    int e = e2 - 1;                     /* |x| in [2^e, 2^(e+1)) */
+    if (e < -126) e = -126;             /* subnormal range: fixed quantum */
+    double quantum = ldexp(1.0, e - 7);
+    double y = rint(x / quantum) * quantum;
+    if (fabs(y) >= ldexp(1.0, 128))     /* rounded past the largest finite */
+        return y > 0 ? 0x7F80u : 0xFF80u;
+    float f = (float)y;                 /* exact: y has <= 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(u >> 16);
+}
+
+void wfo_bf16_to_f64(const uint16_t *in, double *out, long n)
+{
+    for (long i = 0; i < n; ++i) out[i] = bf16_bits_to_double(in[i]);
+}
+
+void wfo_f64_to_bf16(const double *in, uint16_t *out, long n)
+{
+    for (long i = 0; i < n; ++i) out[i] = double_to_bf16_bits(in[i]);
+}
+
+/* ---- positions ------------------------------------------------------------ */
+
+void wfo_positions(long round, int n_wave, int F, int gh, int gw, int32_t *pos)
+{
+    const int L = F * gh * gw;
+    for (int c = 0; c < n_wave; ++c) {
+        long g = round + c;
+        for (int f = 0; f < F; ++f)
+            for (int y = 0; y < gh; ++y)
+                for (int x = 0; x < gw; ++x) {
+                    long n = (long)c * L + (long)f * gh * gw + (long)y * gw + x;
+                    pos[3 * n + 0] = (int32_t)(g * F + f);
+                    pos[3 * n + 1] = y;
+                    pos[3 * n + 2] = x;
+                }
+    }
+}
+
+/* ---- RMSNorm and RoPE on one head vector -------------------------------- */
+
+void wfo_rms_norm(const double *x, const double *gamma, int D, double eps, double *y)
+{
+    double ss = 0.0;
+    for (int d = 0; d < D; ++d) ss += x[d] * x[d];
+    double inv = 1.0 / sqrt(ss / D + eps);
+    for (int d = 0; d < D; ++d) y[d] = x[d] * inv * gamma[d];
+}
+
+void wfo_rope_3d(const double *x, int D, int dt, int dh, int dw, double theta,
+                 const int32_t *pos_thw, double *y)
+{
+    const int width[3] = {dt, dh, dw};
+    int off = 0;
+    for (int a = 0; a < 3; ++a) {
+        const int da = width[a];
+        for (int i = 0; i < da / 2; ++i) {
+            double omega = pow(theta, -2.0 * i / (double)da);
+            double phi = (double)pos_thw[a] * omega;
+            double cs = cos(phi), sn = sin(phi);
+            double x0 = x[off + 2 * i], x1 = x[off + 2 * i + 1];
+            y[off + 2 * i]     = x0 * cs - x1 * sn;
+            y[off + 2 * i + 1] = x0 * sn + x1 * cs;
+        }
+        off += da;
+    }
+    (void)D;
+}
+
+/* ---- fused append (norm + rope + bf16 rounding) ------------------------- */
+
+int wfo_append(int T, int H, int D,
+               const uint16_t *q, const uint16_t *k, const uint16_t *v,
+               const int32_t *pos,                 /* [T,3] */
+               const float *gamma_q, const float *gamma_k,   /* [H,D] */
+               double eps, int dt, int dh, int dw, double theta,
+               uint16_t *q_out, uint16_t *k_out, uint16_t *v_out,  /* [T,H,D] */
+               double *q_f64, double *k_f64)       /* [T,H,D] or NULL */
+{
+    if (dt + dh + dw != D || (dt | dh | dw) & 1) return -1;
+    const long rows = (long)T * H;
+#pragma omp parallel
+    {
+        double *xin = (double *)malloc(sizeof(double) * D);
+        double *gam = (double *)malloc(sizeof(double) * D);
+        double *nrm = (double *)malloc(sizeof(double) * D);
+        double *rot = (double *)malloc(sizeof(double) * D);
+#pragma omp for schedule(static)
+        for (long row = 0; row < rows; ++row) {
+            const long n = row / H, h = row % H;
+            const long base = row * D;
+            for (int which = 0; which < 2; ++which) {
+                const uint16_t *src = which ? k : q;
+                const float *g = which ? gamma_k : gamma_q;
+                uint16_t *dst = which ? k_out : q_out;
+                double *dst64 = which ? k_f64 : q_f64;
+                for (int d = 0; d < D; ++d) {
+                    xin[d] = bf16_bits_to_double(src[base + d]);
+                    gam[d] = (double)g[h * D + d];
+                }
+                wfo_rms_norm(xin, gam, D, eps, nrm);
+                wfo_rope_3d(nrm, D, dt, dh, dw, theta, pos + 3 * n, rot);
+                for (int d = 0; d < D; ++d) {
+                    dst[base + d] = double_to_bf16_bits(rot[d]);
+                    if (dst64) dst64[base + d] = rot[d];
+                }
+            }
+            for (int d = 0; d < D; ++d) v_out[base + d] = v[base + d];
+        }
+        free(xin); free(gam); free(nrm); free(rot);
+    }
+    return 0;
+}
+
+/* ---- chunk-causal attention on selected rows ----------------------------- */
+
+/*
+ * q       : [Tq, H, D] bf16 bits, the queries (wave tokens, already normed/roped)
+ * q_chunk : absolute chunk id of every query chunk; query n lies in chunk n / L
+ * kv      : k, v as [n_kchunks * L, H, D] bf16 bits, chunk b holds rows [b*L, (b+1)*L)
+ * k_chunk : absolute chunk id of every key chunk
+ * rows, heads : the n_sel (query row, head) pairs to compute
+ * o       : [n_sel, D] doubles; lse : [n_sel] natural-log sum-exp (may be NULL)
+ */
+int wfo_chunk_causal_attn_rows(int H, int D, int L,
+                               const uint16_t *q, const int64_t *q_chunk,
+                               const uint16_t *k, const uint16_t *v,
+                               const int64_t *k_chunk, int n_kchunks,
+                               int n_sel, const int32_t *rows, const int32_t *heads,
+                               double *o, double *lse)
+{
+    const long nk = (long)n_kchunks * L;
+    const double scale = 1.0 / sqrt((double)D);
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *qd = (double *)malloc(sizeof(double) * D);
+        double *s = (double *)malloc(sizeof(double) * (nk > 0 ? nk : 1));
+        unsigned char *vis = (unsigned char *)malloc(nk > 0 ? nk : 1);
+        double *acc = (double *)malloc(sizeof(double) * D);
+#pragma omp for schedule(dynamic, 1)
+        for (int i = 0; i < n_sel; ++i) {
+            const long n = rows[i];
+            const int h = heads[i];
+            const int64_t qid = q_chunk[n / L];
+            for (int d = 0; d < D; ++d)
+                qd[d] = bf16_bits_to_double(q[(n * H + h) * D + d]);
+            double m = -INFINITY;
+            long nvis = 0;
+            for (long j = 0; j < nk; ++j) {
+                vis[j] = k_chunk[j / L] <= qid;
+                if (!vis[j]) continue;
+                double dot = 0.0;
+                for (int d = 0; d < D; ++d)
+                    dot += qd[d] * bf16_bits_to_double(k[(j * H + h) * D + d]);
+                s[j] = dot * scale;
+                if (s[j] > m) m = s[j];
+                ++nvis;
+            }
+            if (nvis == 0) {
+#pragma omp atomic write
+                bad = 1;
+                continue;
+            }
+            double z = 0.0;
+            for (int d = 0; d < D; ++d) acc[d] = 0.0;
+            for (long j = 0; j < nk; ++j) {
+                if (!vis[j]) continue;
+                double w = exp(s[j] - m);
+                z += w;
+                for (int d = 0; d < D; ++d)
+                    acc[d] += w * bf16_bits_to_double(v[(j * H + h) * D + d]);
+            }
+            for (int d = 0; d < D; ++d) o[(long)i * D + d] = acc[d] / z;
+            if (lse) lse[i] = m + log(z);
+        }
+        free(qd); free(s); free(vis); free(acc);
+    }
+    return bad ? -2 : 0;
+}
+
+int wfo_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
