@@ -1,0 +1,452 @@
+"""Benchmark of the wave-round hot path on B200: fused append + chunk-causal attention.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one wave round of one layer: wf_qk_norm_rope_append (per-head Q/K
+RMSNorm, 3D RoPE, K/V into the ring) followed by wf_chunk_causal_attn, with
+the ring advancing one chunk per step (steady state, full history).  Inputs
+are seeded synthetic bf16 N(0,1) tensors resident in HBM before timing.
+
+Prints ONE JSON line (rank 0).  `value` is useful attention TFLOP/s over all
+ranks (QK^T + PV over visible, unpadded query/key pairs / step time).  Under
+torchrun every rank runs its own replica of the workload on its own GPU (the
+path shards by independent problems; no data-path collective).
+
+--impl reference times the fp64 CPU oracle (the parity reference) on a
+bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from chunk_causal_dit_b200 import inputs as wi  # noqa: E402
+
+METRIC = "wave-round chunk-causal attention useful TFLOP/s & chunks/s on 1 B200; % of peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+BAD_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for name in ("attn_kernel.cu", "sm100.cuh", "wf_internal.h"):
+        with open(os.path.join(ROOT, "chunk_causal_dit_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload):
+    """Per-launch DRAM bytes of the attention kernel from the committed ncu summary,
+    or None when the summary is missing or was taken on another kernel source."""
+    path = os.path.join(ROOT, "profiles", "attn_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    if d.get("kernel_hash") != kernel_source_hash():
+        return None
+    return d.get("per_launch_bytes", {}).get(workload)
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples with host timestamps."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.proc = None
+        self.lines = []
+        self.gpu = gpu_index
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self, t0, t1):
+        import datetime
+        samples = []
+        for ln in self.lines:
+            p = [x.strip() for x in ln.split(",")]
+            if len(p) < 10:
+                continue
+            try:
+                ts = datetime.datetime.strptime(p[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                continue
+            samples.append((ts, p))
+        inside = [s for s in samples if t0 - 0.05 <= s[0] <= t1 + 0.05] or samples
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(p[2]) for _, p in inside if p[2].replace(".", "").isdigit()]
+        mx = [float(p[3]) for _, p in inside if p[3].replace(".", "").isdigit()]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for _, p in inside for n, v in zip(names, p[6:10]) if v == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(inside), "power_w_max": max(
+                    (float(p[4]) for _, p in inside if p[4].replace(".", "").isdigit()),
+                    default=None)}
+
+
+def dist_setup(gpus):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != gpus and world > 1:
+        raise SystemExit("--gpus %d but WORLD_SIZE %d" % (gpus, world))
+    return rank, world, local
+
+
+def make_group(world, backend):
+    import datetime
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist if world > 1 else None
+
+
+def barrier(dist, device=None):
+    if dist is not None:
+        if device is not None:
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def allreduce_max(dist, value, device):
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ ours --
+
+def run_ours(args, rank, world, local):
+    import torch
+    from chunk_causal_dit_b200 import wf
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = make_group(world, "nccl")
+    w = wi.WORKLOADS[args.workload]
+    peaks, peak_src = load_peaks()
+
+    plan = wf.Plan(w.L, w.n_wave, w.n_hist, w.H, w.D).set_rope(w.F, w.gh, w.gw)
+    x = wi.wave_inputs(w, seed=rank)
+    hk, hv = wi.history_prefill(w, seed=rank)
+    q, k, v = x.q.to(dev), x.k.to(dev), x.v.to(dev)
+    gq, gk = x.gamma_q.to(dev), x.gamma_k.to(dev)
+    kc = torch.empty((w.R, w.L, w.H, w.D), dtype=torch.bfloat16, device=dev)
+    vc = torch.empty_like(kc)
+    for j in range(w.n_hist):
+        kc[j % w.R].copy_(hk[j])
+        vc[j % w.R].copy_(hv[j])
+    q_out = torch.empty_like(q)
+    o = torch.empty_like(q)
+    stream = torch.cuda.current_stream(dev)
+    r0 = w.n_hist
+    flops_step = wf.wf_useful_flops(plan, r0)
+    tensor_bytes = w.T * w.H * w.D * 2
+    append_bytes = 12 * w.T * w.H * w.D
+
+    def step(r):
+        wf.wf_qk_norm_rope_append(plan, r, q, k, v, None, gq, gk, q_out, kc, vc, stream)
+        wf.wf_chunk_causal_attn(plan, r, q_out, kc, vc, o, None, stream)
+
+    rnd = r0
+    for _ in range(args.warmup):
+        step(rnd)
+        rnd += 1
+    torch.cuda.synchronize(dev)
+    if wf.wf_sync_status(plan, stream) != wf.WF_OK:
+        raise SystemExit("device status error during warm-up")
+
+    # ---- device-timed steps (kernel events inside give the roofline) ----
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local) if rank == 0 or True else None
+    time.sleep(0.3)
+    barrier(dist, dev)
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    start.record(stream)
+    for i in range(args.steps):
+        e0, e1, e2 = ev[i]
+        e0.record(stream)
+        wf.wf_qk_norm_rope_append(plan, rnd, q, k, v, None, gq, gk, q_out, kc, vc, stream)
+        e1.record(stream)
+        wf.wf_chunk_causal_attn(plan, rnd, q_out, kc, vc, o, None, stream)
+        e2.record(stream)
+        rnd += 1
+    stop.record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    barrier(dist, dev)
+    clocks.stop()
+    status = wf.wf_sync_status(plan, stream)
+    if status != wf.WF_OK:
+        raise SystemExit("device status %d (%s)" % (status, wf.status_string(status)))
+    ms_total = allreduce_max(dist, start.elapsed_time(stop), dev)
+    ms_step = ms_total / args.steps
+    t_append = [a.elapsed_time(b) for a, b, _ in ev]
+    t_attn = [b.elapsed_time(c) for _, b, c in ev]
+    attn_ms = statistics.mean(t_attn)
+    append_ms = statistics.mean(t_append)
+
+    # ---- end to end through the API: pinned host in, pinned host out ----
+    hq = x.q.pin_memory()
+    hk_ = x.k.pin_memory()
+    hv_ = x.v.pin_memory()
+    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    e2e_steps = max(3, min(args.steps, 50))
+
+    def e2e_step(r):
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk_, non_blocking=True)
+        v.copy_(hv_, non_blocking=True)
+        step(r)
+        ho.copy_(o, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step(rnd)
+        rnd += 1
+    barrier(dist, dev)
+    torch.cuda.synchronize(dev)
+    s2, t2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step(rnd)
+        rnd += 1
+    t2.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = allreduce_max(dist, s2.elapsed_time(t2), dev) / e2e_steps
+    barrier(dist, dev)
+
+    clk = clocks.summary(t_wall0, t_wall1)
+    plan.destroy()
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+
+    peak_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    attn_tflops = flops_step / (attn_ms * 1e-3) / 1e12
+    value = world * flops_step / (ms_step * 1e-3) / 1e12
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    append_gbs = append_bytes / (append_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded bf16 N(0,1) q/k/v and history, gains 1+0.1N(0,1))",
+        "config": {
+            "workload": w.name,
+            "heads": w.H, "head_dim": w.D, "chunk_tokens": w.L, "wave_chunks": w.n_wave,
+            "history_chunks": w.n_hist, "wave_tokens": w.T,
+            "parallelism": "replica%d (independent wave rounds, no data-path collective)" % world,
+            "l2": "no flush: per-step working set %.0f MB > 126 MB L2" % (
+                (append_bytes + 2 * w.R * w.L * w.H * w.D * 2) / 1e6),
+        },
+        "chunks_per_s": round(world * w.n_wave / (ms_step * 1e-3), 2),
+        "pct_peak": round(100.0 * value / world / peak_tf, 2),
+        "roofline": {
+            "kernel": "chunk_causal_attn_kernel",
+            "bound": "tensor",
+            "achieved": round(attn_tflops, 2),
+            "peak": peak_tf,
+            "unit": "TFLOP/s",
+            "frac": round(attn_tflops / peak_tf, 4),
+            "peak_source": "%s bf16_tflops (burst)" % peak_src,
+            "traffic": profiled_traffic(args.workload),
+            "ms_per_launch": round(attn_ms, 5),
+            "useful_flop_per_launch": flops_step,
+        },
+        "append": {
+            "kernel": "qk_norm_rope_append_kernel",
+            "bound": "hbm",
+            "ms_per_launch": round(append_ms, 5),
+            "achieved": round(append_gbs, 1),
+            "peak": hbm,
+            "unit": "GB/s",
+            "frac": round(append_gbs / hbm, 4),
+            "bytes_per_launch": append_bytes,
+        },
+        "e2e": {
+            "value": round(world * flops_step / (e2e_ms * 1e-3) / 1e12, 3),
+            "unit": "TFLOP/s",
+            "ms_per_step": round(e2e_ms, 4),
+            "h2d_bytes_per_step": 3 * tensor_bytes,
+            "d2h_bytes_per_step": tensor_bytes,
+        },
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
+    return line
+
+
+# --------------------------------------------------------- oracle (CPU) --
+
+def oracle_round_setup(w, seed=0):
+    """Host inputs of one steady-state round (round = n_hist) through the oracle."""
+    import oracle
+    r = w.n_hist
+    x = wi.wave_inputs(w, seed=seed)
+    hk, hv = wi.history_prefill(w, seed=seed)
+    pos = oracle.positions(r, w.n_wave, w.F, w.gh, w.gw)
+    qo, ko, vo = oracle.append(wi.bits(x.q), wi.bits(x.k), wi.bits(x.v), pos,
+                               x.gamma_q.numpy(), x.gamma_k.numpy())
+    cache = oracle.OracleCache(w.L)
+    for j in range(w.n_hist):
+        cache.put(j, wi.bits(hk[j]), wi.bits(hv[j]))
+    cache.put_wave(r, ko, vo)
+    k, v, ids = cache.round_keys(r, w.n_wave, w.n_hist)
+    return r, qo, k, v, ids
+
+
+def oracle_sample_step(w, r, qo, k, v, ids, n_pairs, rng):
+    import oracle
+    rows = rng.integers(0, w.T, n_pairs)
+    heads = rng.integers(0, w.H, n_pairs)
+    qids = np.arange(r, r + w.n_wave)
+    t0 = time.perf_counter()
+    oracle.chunk_causal_attn_rows(qo, qids, k, v, ids, w.L, rows, heads, want_lse=False)
+    dt = time.perf_counter() - t0
+    hv = min(w.n_hist, r)
+    flops = float(sum(4.0 * w.D * (hv + row // w.L + 1) * w.L for row in rows))
+    return flops, dt
+
+
+def cpu_baseline(w, budget_s=15.0):
+    import oracle
+    r, qo, k, v, ids = oracle_round_setup(w)
+    rng = np.random.default_rng(0)
+    flops, secs = 0.0, 0.0
+    n = 16
+    while secs < budget_s:
+        f, dt = oracle_sample_step(w, r, qo, k, v, ids, n, rng)
+        flops += f
+        secs += dt
+        n = min(4096, n * 2)
+    return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s",
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": "%.0f s of fp64 oracle attention on random (row, head) pairs of the "
+                      "same round (%.3g useful FLOP)" % (secs, flops)}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    import oracle
+    w = wi.WORKLOADS[args.workload]
+    r, qo, k, v, ids = oracle_round_setup(w)
+    rng = np.random.default_rng(1)
+    pairs = args.ref_pairs
+    for _ in range(args.warmup):
+        oracle_sample_step(w, r, qo, k, v, ids, pairs, rng)
+    flops, secs = 0.0, 0.0
+    for _ in range(args.steps):
+        f, dt = oracle_sample_step(w, r, qo, k, v, ids, pairs, rng)
+        flops += f
+        secs += dt
+    value = flops / secs / 1e12
+    sample = ("each step: fp64 oracle attention of %d random (row, head) pairs of the round "
+              "(all their visible keys)" % pairs)
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 6),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(1e3 * secs / args.steps, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded, same generator as the GPU arm)",
+        "config": {"workload": w.name, "heads": w.H, "head_dim": w.D, "chunk_tokens": w.L,
+                   "wave_chunks": w.n_wave, "history_chunks": w.n_hist},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s",
+                         "cores": oracle.num_threads(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="wan13b_4step", choices=sorted(wi.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--ref-pairs", type=int, default=48)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    rank, world, local = dist_setup(args.gpus)
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+    else:
+        line = run_ours(args, rank, world, local)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,438 @@
+// attn_kernel.cu -- chunk-causal wave-round attention on sm_100a tensor cores.
+//
+// "Wave Forcing" (abstract): chunk-wise causal attention lets each chunk of the
+// wave read earlier, cleaner chunks before their denoising is complete.  For
+// query chunk c the visible keys are every token of the valid history chunks
+// and of wave chunks 0..c; inside a chunk attention is bidirectional.  Visible
+// keys therefore form whole chunks, so masking is decided per key tile: fully
+// masked tiles are never loaded, and the only element mask is "key row < L" in
+// the last 128-key tile of each chunk (TMA fills the rows past L with zeros).
+//
+// Work unit = (wave chunk c, head h, pair of 128-row query tiles).  One CTA per
+// SM walks units in longest-first order (cost (h_valid + c + 1) key chunks).
+// Warp roles (320 threads):
+//   warps 0-3  softmax for query tile 0 (TMEM lanes 0..127, one row per thread)
+//   warps 4-7  softmax for query tile 1
+//   warp  8    TMA producer: Q tiles, then K_j, V_j into a ring of smem stages
+//   warp  9    MMA issuer (one thread): S_x = Q_x K_j^T, O_x += P_x V_j
+// TMEM (512 columns): S0 | S1 | O0 | O1.  Softmax overwrites the first half of
+// S_x with P_x (bf16 pairs) and the PV product reads P straight from TMEM.
+// The two query tiles ping-pong: while one warpgroup exponentiates, the tensor
+// core runs the other tile's PV and next QK^T.  Online softmax works in the
+// log2 domain and rescales O only when a row maximum grows by more than 2^8.
+//
+// Every mbarrier wait is bounded (clock64 limit); on expiry the kernel records
+// kStatusTimeout in the plan's status word, all roles leave their loops, wait
+// for their own copies/MMAs in flight, and the CTA frees TMEM and returns.
+#include <cuda_bf16.h>
+
+#include "sm100.cuh"
+#include "wf_internal.h"
+
+namespace wf {
+
+namespace {
+
+constexpr int BM = 128;              // query rows per tile
+constexpr int BN = 128;              // keys per tile
+constexpr int kThreads = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units
+
+template <int D>
+struct Cfg {
+    static constexpr int kStages = D == 128 ? 4 : 8;
+    static constexpr int kHalves = D / 64;                 // 128-byte column blocks
+    static constexpr uint32_t kHalfBytes = 128 * 128;      // 128 rows x 128 bytes
+    static constexpr uint32_t kTileBytes = BM * D * 2;
+    static constexpr uint32_t kQOff = 0;
+    static constexpr uint32_t kKVOff = 2 * kTileBytes;
+    static constexpr uint32_t kBarOff = kKVOff + kStages * kTileBytes;
+    static constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;
+    static constexpr uint32_t kS0 = 0, kS1 = 128, kO0 = 256, kO1 = 256 + D;
+};
+
+// Barrier indices inside the barrier block (8 bytes each).
+template <int S>
+struct Bars {
+    static constexpr int q_full = 0, q_empty = 1, s_full = 2, p_ready = 4, o_final = 6,
+                         drain = 8, kv_full = 9, kv_empty = 9 + S, count = 9 + 2 * S;
+};
+
+// Wait-site codes recorded in DeviceWords::timeout_where.
+enum : uint32_t {
+    kWhereProducerQ = 1, kWhereProducerKV = 2, kWhereMmaQ = 3, kWhereMmaKV = 4,
+    kWhereMmaP = 5, kWhereSoftS = 6, kWhereSoftO = 7, kWhereDrain = 8,
+};
+
+struct Ctl {
+    volatile uint32_t *abort;
+    DeviceWords *words;
+    unsigned long long limit;
+};
+
+// Bounded wait on one mbarrier phase.  Returns false on timeout or when another
+// role already aborted (unless `drain`, which ignores the abort flag).
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ctl &ctl,
+                                         uint32_t where, bool drain = false)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+#pragma unroll 1
+        for (int k = 0; k < 32; ++k)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (!drain && *ctl.abort) return false;
+        if (static_cast<unsigned long long>(clock64() - t0) > ctl.limit) {
+            *ctl.abort = 1u;
+            atomicOr(&ctl.words->status, kStatusTimeout);
+            atomicCAS(&ctl.words->timeout_where, 0u, where);
+            return false;
+        }
+    }
+}
+
+struct Unit {
+    int c, h, pair, n_kt;
+};
+
+__device__ __forceinline__ Unit decode_unit(const AttnParams &p, int u)
+{
+    Unit r;
+    const int per_c = p.H * p.n_qpairs;
+    const int ci = u / per_c;
+    const int rem = u - ci * per_c;
+    r.c = p.W - 1 - ci;                       // longest (latest chunk) first
+    r.h = rem / p.n_qpairs;
+    r.pair = rem - r.h * p.n_qpairs;
+    r.n_kt = (p.h_valid + r.c + 1) * p.n_ktiles;
+    return r;
+}
+
+template <int D>
+__device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t q_smem, uint32_t k_smem)
+{
+    constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, false);
+#pragma unroll
+    for (int s = 0; s < D / 16; ++s) {
+        const uint32_t off = (s >> 2) * Cfg<D>::kHalfBytes + (s & 3) * 32;
+        umma_ss(s_tmem, sw128_desc(q_smem + off, 16, 1024), sw128_desc(k_smem + off, 16, 1024),
+                idesc, s > 0 ? 1u : 0u);
+    }
+}
+
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem,
+                                         bool accumulate)
+{
+    constexpr uint32_t idesc = idesc_bf16_f32(BM, D, true);
+#pragma unroll
+    for (int s = 0; s < BN / 16; ++s) {
+        // V tile: 16 keys per step = 2 eight-row groups of 128 bytes; the two
+        // 64-channel halves of D sit kHalfBytes apart (leading byte offset).
+        umma_ts(o_tmem, p_tmem + s * 8, sw128_desc(v_smem + s * 2048, Cfg<D>::kHalfBytes, 1024),
+                idesc, (accumulate || s > 0) ? 1u : 0u);
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                         const __grid_constant__ CUtensorMap tmap_k,
+                         const __grid_constant__ CUtensorMap tmap_v,
+                         const AttnParams p)
+{
+    using C = Cfg<D>;
+    constexpr int S = C::kStages;
+    using B = Bars<S>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = smem_addr(smem);
+    const uint32_t sq = sbase + C::kQOff;
+    const uint32_t skv = sbase + C::kKVOff;
+    const uint32_t sbar = sbase + C::kBarOff;
+    auto bar = [&](int i) -> uint32_t { return sbar + 8u * static_cast<uint32_t>(i); };
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kBarOff + 8 * B::count);
+    volatile uint32_t *abort_flag = tmem_slot + 1;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(B::q_full), 1);
+        mbar_init(bar(B::q_empty), 1);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(bar(B::s_full + x), 1);
+            mbar_init(bar(B::p_ready + x), 128);
+            mbar_init(bar(B::o_final + x), 1);
+        }
+        mbar_init(bar(B::drain), 1);
+        for (int s = 0; s < S; ++s) {
+            mbar_init(bar(B::kv_full + s), 1);
+            mbar_init(bar(B::kv_empty + s), 1);
+        }
+        *abort_flag = 0u;
+        fence_barrier_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const Ctl ctl{abort_flag, p.words, p.wait_limit};
+
+    if (warp == kProducerWarp) {
+        if (lane == 0) {
+            tma_prefetch_desc(&tmap_q);
+            tma_prefetch_desc(&tmap_k);
+            tma_prefetch_desc(&tmap_v);
+            uint32_t stage = 0, kv_phase = 0, q_phase = 0;
+            uint32_t q_fills = 0, kv_fills = 0;   // copies issued so far
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < p.n_units; u += gridDim.x) {
+                const Unit un = decode_unit(p, u);
+                if (!(ok = wait_bar(bar(B::q_empty), q_phase ^ 1u, ctl, kWhereProducerQ))) break;
+                q_phase ^= 1u;
+                mbar_arrive_expect_tx(bar(B::q_full), 2 * C::kTileBytes);
+                ++q_fills;
+                for (int x = 0; x < 2; ++x)
+                    for (int hf = 0; hf < C::kHalves; ++hf)
+                        tma_load_4d(sq + x * C::kTileBytes + hf * C::kHalfBytes, &tmap_q,
+                                    bar(B::q_full), hf * 64, un.h, (2 * un.pair + x) * BM, un.c);
+                for (int j = 0; ok && j < un.n_kt; ++j) {
+                    const int b = j / p.n_ktiles;
+                    const int t = j - b * p.n_ktiles;
+                    const int slot = ring_slot(visible_chunk_id(p.round, p.h_valid, b), p.R);
+                    for (int kv = 0; kv < 2; ++kv) {
+                        if (!(ok = wait_bar(bar(B::kv_empty + stage), kv_phase ^ 1u, ctl,
+                                            kWhereProducerKV)))
+                            break;
+                        mbar_arrive_expect_tx(bar(B::kv_full + stage), C::kTileBytes);
+                        ++kv_fills;
+                        const CUtensorMap *map = kv ? &tmap_v : &tmap_k;
+                        for (int hf = 0; hf < C::kHalves; ++hf)
+                            tma_load_4d(skv + stage * C::kTileBytes + hf * C::kHalfBytes, map,
+                                        bar(B::kv_full + stage), hf * 64, un.h, t * BN, slot);
+                        if (++stage == S) { stage = 0; kv_phase ^= 1u; }
+                    }
+                }
+            }
+            if (!ok) {
+                // let every copy already issued land before the CTA releases smem
+                if (q_fills) wait_bar(bar(B::q_full), (q_fills - 1) & 1u, ctl, kWhereDrain, true);
+                for (uint32_t s = 0; s < static_cast<uint32_t>(S); ++s) {
+                    const uint32_t f = (kv_fills + S - 1 - s) / S;   // fills of stage s
+                    if (f) wait_bar(bar(B::kv_full + s), (f - 1) & 1u, ctl, kWhereDrain, true);
+                }
+            }
+        }
+    } else if (warp == kMmaWarp) {
+        if (lane == 0) {
+            uint32_t stage = 0, kv_phase = 0, q_phase = 0;
+            uint32_t p_phase[2] = {0u, 0u};
+            const uint32_t tS[2] = {tmem + C::kS0, tmem + C::kS1};
+            const uint32_t tO[2] = {tmem + C::kO0, tmem + C::kO1};
+            const uint32_t sQ[2] = {sq, sq + C::kTileBytes};
+            bool ok = true;
+            // take the next K/V stage in ring order, waiting until its copy landed
+#define WF_NEXT_STAGE(st)                                                              \
+    ((st) = stage,                                                                     \
+     ok = wait_bar(bar(B::kv_full + stage), kv_phase, ctl, kWhereMmaKV),               \
+     (++stage == S ? (stage = 0, kv_phase ^= 1u) : 0u), tc_fence_after(), ok)
+            for (int u = blockIdx.x; ok && u < p.n_units; u += gridDim.x) {
+                const Unit un = decode_unit(p, u);
+                if (!(ok = wait_bar(bar(B::q_full), q_phase, ctl, kWhereMmaQ))) break;
+                q_phase ^= 1u;
+                uint32_t kst;
+                if (!WF_NEXT_STAGE(kst)) break;
+                issue_qk<D>(tS[0], sQ[0], skv + kst * C::kTileBytes);
+                umma_commit(bar(B::s_full + 0));
+                issue_qk<D>(tS[1], sQ[1], skv + kst * C::kTileBytes);
+                umma_commit(bar(B::s_full + 1));
+                umma_commit(bar(B::kv_empty + kst));
+                if (un.n_kt == 1) umma_commit(bar(B::q_empty));
+                for (int j = 0; ok && j < un.n_kt; ++j) {
+                    const bool more = j + 1 < un.n_kt;
+                    uint32_t vst, kst2 = 0;
+                    if (!WF_NEXT_STAGE(vst)) break;
+                    // query tile 0
+                    if (!(ok = wait_bar(bar(B::p_ready + 0), p_phase[0], ctl, kWhereMmaP))) break;
+                    p_phase[0] ^= 1u;
+                    tc_fence_after();
+                    issue_pv<D>(tO[0], tS[0], skv + vst * C::kTileBytes, j > 0);
+                    if (more) {
+                        if (!WF_NEXT_STAGE(kst2)) break;
+                        issue_qk<D>(tS[0], sQ[0], skv + kst2 * C::kTileBytes);
+                        umma_commit(bar(B::s_full + 0));
+                    } else {
+                        umma_commit(bar(B::o_final + 0));
+                    }
+                    // query tile 1
+                    if (!(ok = wait_bar(bar(B::p_ready + 1), p_phase[1], ctl, kWhereMmaP))) break;
+                    p_phase[1] ^= 1u;
+                    tc_fence_after();
+                    issue_pv<D>(tO[1], tS[1], skv + vst * C::kTileBytes, j > 0);
+                    umma_commit(bar(B::kv_empty + vst));
+                    if (more) {
+                        issue_qk<D>(tS[1], sQ[1], skv + kst2 * C::kTileBytes);
+                        umma_commit(bar(B::s_full + 1));
+                        umma_commit(bar(B::kv_empty + kst2));
+                        if (j + 2 == un.n_kt) umma_commit(bar(B::q_empty));
+                    } else {
+                        umma_commit(bar(B::o_final + 1));
+                    }
+                }
+            }
+#undef WF_NEXT_STAGE
+            // every MMA issued by this thread completes before TMEM is released
+            umma_commit(bar(B::drain));
+            wait_bar(bar(B::drain), 0u, ctl, kWhereDrain, true);
+        }
+    } else {
+        // ---------------- softmax warpgroups ----------------
+        const int x = warp >> 2;                    // query tile of this warpgroup
+        const int row = threadIdx.x & 127;          // TMEM lane = row of the tile
+        const uint32_t lane_sel = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + lane_sel + (x ? C::kS1 : C::kS0);
+        const uint32_t tO = tmem + lane_sel + (x ? C::kO1 : C::kO0);
+        const float scale = p.scale_log2;
+        uint32_t s_phase = 0, o_phase = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; ok && u < p.n_units; u += gridDim.x) {
+            const Unit un = decode_unit(p, u);
+            const int q_row = (2 * un.pair + x) * BM + row;     // row inside chunk c
+            float m_run = -INFINITY, l_run = 0.f;
+            for (int j = 0; j < un.n_kt; ++j) {
+                ok = wait_bar(bar(B::s_full + x), s_phase, ctl, kWhereSoftS);
+                ok = __all_sync(0xFFFFFFFFu, ok);
+                if (!ok) break;
+                s_phase ^= 1u;
+                tc_fence_after();
+                uint32_t r[4][32];
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tS + q4 * 32, r[q4]);
+                tmem_wait_ld();
+                const int t = j % p.n_ktiles;
+                const int valid = t == p.n_ktiles - 1 ? p.L - t * BN : BN;
+                float mx = -INFINITY;
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        float s = __uint_as_float(r[q4][e]);
+                        if (q4 * 32 + e >= valid) s = -INFINITY;
+                        r[q4][e] = __float_as_uint(s);
+                        mx = fmaxf(mx, s);
+                    }
+                // The row maximum only moves forward when it grew by more than
+                // 2^8: otherwise exponents stay <= 2^8 against the stale maximum
+                // and O keeps its scale.  (At j = 0 PV overwrites O.)
+                const float m_new = fmaxf(m_run, mx * scale);
+                const bool need = m_new > m_run + kRescaleThreshold;
+                const float alpha = need ? ex2_approx(m_run - m_new) : 1.0f;
+                if (need) {
+                    l_run *= alpha;
+                    m_run = m_new;
+                }
+                const float neg_m = -m_run;
+                float sum = 0.f;
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    // P columns [64*hf, 64*hf + 64) -> packed bf16 TMEM columns [32*hf, 32*hf + 32)
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int col = 64 * hf + 2 * e;
+                        const float p0 = ex2_approx(fmaf(__uint_as_float(r[col >> 5][col & 31]), scale, neg_m));
+                        const float p1 = ex2_approx(fmaf(__uint_as_float(r[col >> 5][(col + 1) & 31]), scale, neg_m));
+                        sum += p0 + p1;
+                        pk[e] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st32(tS + 32 * hf, pk);
+                }
+                l_run += sum;
+                if (j > 0 && __any_sync(0xFFFFFFFFu, need)) {
+                    // O is quiescent here: the MMA that filled S_x(j) was issued
+                    // after PV_x(j-1), and PV_x(j) waits for this warpgroup.
+#pragma unroll 1
+                    for (int cc = 0; cc < D / 32; ++cc) {
+                        uint32_t o[32];
+                        tmem_ld32(tO + cc * 32, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tmem_st32(tO + cc * 32, o);
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(B::p_ready + x));
+            }
+            if (!ok) break;
+            ok = wait_bar(bar(B::o_final + x), o_phase, ctl, kWhereSoftO);
+            ok = __all_sync(0xFFFFFFFFu, ok);
+            if (!ok) break;
+            o_phase ^= 1u;
+            tc_fence_after();
+            const float inv_l = 1.0f / l_run;
+            const bool store = q_row < p.L;
+            const long n = static_cast<long>(un.c) * p.L + q_row;
+            uint16_t *dst = p.o + (n * p.H + un.h) * D;
+#pragma unroll 1
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t o[32];
+                tmem_ld32(tO + cc * 32, o);
+                tmem_wait_ld();
+                uint4 w[4];
+                uint32_t *wp = reinterpret_cast<uint32_t *>(w);
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    wp[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l,
+                                        __uint_as_float(o[2 * e + 1]) * inv_l);
+                if (store) {
+                    uint4 *d4 = reinterpret_cast<uint4 *>(dst + cc * 32);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) d4[e] = w[e];
+                }
+            }
+            if (store && p.lse != nullptr)
+                p.lse[static_cast<long>(un.h) * p.T + n] = m_run * 0.6931471805599453f + logf(l_run);
+            tc_fence_before();
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace
+
+template <int D>
+static cudaError_t launch_attn_d(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                                 const AttnParams &p, int grid, cudaStream_t stream)
+{
+    const uint32_t smem = Cfg<D>::kSmemBytes;
+    cudaError_t e = cudaFuncSetAttribute(chunk_causal_attn_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    chunk_causal_attn_kernel<D><<<grid, kThreads, smem, stream>>>(mq, mk, mv, p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_attn(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                        const AttnParams &p, int D, int grid, cudaStream_t stream)
+{
+    return D == 128 ? launch_attn_d<128>(mq, mk, mv, p, grid, stream)
+                    : launch_attn_d<64>(mq, mk, mv, p, grid, stream);
+}
+
+}  // namespace wf

@@ -1,0 +1,339 @@
+// wf_api.cu -- the C ABI of libwf.so (declared in include/wf.h): plan creation and
+// validation, TMA tensor-map set-up, and the two hot-path launches.
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <new>
+
+#include "wf.h"
+#include "wf_internal.h"
+
+namespace wf {
+cudaError_t launch_append(const AppendParams &p, int D, cudaStream_t stream);
+cudaError_t launch_attn(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                        const AttnParams &p, int D, int grid, cudaStream_t stream);
+}  // namespace wf
+
+namespace {
+
+constexpr unsigned long long kDefaultWaitLimit = 1ull << 32;   // ~2 s of SM clock
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+void fill_rope_table(wf::RopeParams &r, double theta)
+{
+    const int width[3] = {r.dt, r.dh, r.dw};
+    int pair = 0;
+    for (int a = 0; a < 3; ++a)
+        for (int i = 0; i < width[a] / 2; ++i, ++pair) {
+            r.omega[pair] = static_cast<float>(std::pow(theta, -2.0 * i / width[a]));
+            r.axis[pair] = static_cast<int8_t>(a);
+        }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+        else
+            (void)cudaGetLastError();
+    });
+    return fn;
+}
+
+// 4-D map over a [n3][n2][H][D] bf16 tensor (slot/chunk, row, head, channel),
+// box = 64 channels x 1 head x 128 rows x 1 slot, 128-byte swizzle, OOB rows read 0.
+bool encode_map(CUtensorMap *map, const void *base, int D, int H, int n2, int n2_stride_rows,
+                int n3)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
+                                static_cast<cuuint64_t>(n2), static_cast<cuuint64_t>(n3)};
+    const cuuint64_t row = static_cast<cuuint64_t>(H) * D * 2;
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, row,
+                                   row * static_cast<cuuint64_t>(n2_stride_rows)};
+    const cuuint32_t box[4] = {64, 1, 128, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int check_device(const wf_plan_s *p)
+{
+    if (p->device < 0 || p->words == nullptr) return WF_ERR_NO_DEVICE;
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) return WF_ERR_CUDA;
+    if (cur != p->device) return WF_ERR_INVALID_ARG;   // plan belongs to another device
+    if (p->cc_major != 10 || p->cc_minor != 0) return WF_ERR_DEVICE;   // kernels are sm_100a
+    return WF_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int wf_plan(int chunk_tokens, int n_wave_chunks, int n_hist_chunks, int heads, int head_dim,
+            wf_plan_t *out)
+{
+    if (out == nullptr) return WF_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (chunk_tokens < 1 || n_wave_chunks < 1 || n_hist_chunks < 0 || heads < 1)
+        return WF_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return WF_ERR_UNSUPPORTED;
+    const long long T = static_cast<long long>(chunk_tokens) * n_wave_chunks;
+    const long long R = static_cast<long long>(n_hist_chunks) + n_wave_chunks;
+    const long long hd = static_cast<long long>(heads) * head_dim;
+    if (T * hd >= (1ll << 31) || R * chunk_tokens * hd >= (1ll << 40) || R > INT_MAX)
+        return WF_ERR_INVALID_ARG;
+    const long long qtiles = (chunk_tokens + 127) / 128;
+    if (static_cast<long long>(heads) * n_wave_chunks * ((qtiles + 1) / 2) >= INT_MAX)
+        return WF_ERR_INVALID_ARG;
+
+    wf_plan_s *p = new (std::nothrow) wf_plan_s();
+    if (p == nullptr) return WF_ERR_CUDA;
+    p->L = chunk_tokens;
+    p->W = n_wave_chunks;
+    p->Hh = n_hist_chunks;
+    p->H = heads;
+    p->D = head_dim;
+    p->R = static_cast<int>(R);
+    p->theta = 10000.0;
+    p->eps = 1e-6;
+    p->rope.dh = p->rope.dw = 2 * (head_dim / 6);
+    p->rope.dt = head_dim - 2 * p->rope.dh;
+    p->rope.F = p->rope.gh = p->rope.gw = 0;
+    fill_rope_table(p->rope, p->theta);
+    p->wait_limit = kDefaultWaitLimit;
+    p->device = -1;
+    p->num_sms = 0;
+    p->cc_major = p->cc_minor = 0;
+    p->words = nullptr;
+
+    int dev = -1;
+    if (cudaGetDevice(&dev) == cudaSuccess) {
+        int sms = 0, ma = 0, mi = 0;
+        void *w = nullptr;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&ma, cudaDevAttrComputeCapabilityMajor, dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&mi, cudaDevAttrComputeCapabilityMinor, dev) == cudaSuccess &&
+            cudaMalloc(&w, sizeof(wf::DeviceWords)) == cudaSuccess) {
+            if (cudaMemset(w, 0, sizeof(wf::DeviceWords)) == cudaSuccess) {
+                p->device = dev;
+                p->num_sms = sms;
+                p->cc_major = ma;
+                p->cc_minor = mi;
+                p->words = static_cast<wf::DeviceWords *>(w);
+            } else {
+                cudaFree(w);
+            }
+        }
+    }
+    (void)cudaGetLastError();   // a machine without a GPU leaves an error behind
+    *out = p;
+    return WF_OK;
+}
+
+int wf_plan_set_rope(wf_plan_t p, int frames_per_chunk, int grid_h, int grid_w, double theta)
+{
+    if (p == nullptr || frames_per_chunk < 1 || grid_h < 1 || grid_w < 1 || !(theta > 0.0) ||
+        static_cast<long long>(frames_per_chunk) * grid_h * grid_w != p->L)
+        return WF_ERR_INVALID_ARG;
+    p->rope.F = frames_per_chunk;
+    p->rope.gh = grid_h;
+    p->rope.gw = grid_w;
+    p->theta = theta;
+    fill_rope_table(p->rope, theta);
+    return WF_OK;
+}
+
+int wf_plan_set_rope_split(wf_plan_t p, int d_t, int d_h, int d_w)
+{
+    if (p == nullptr || d_t < 0 || d_h < 0 || d_w < 0 || ((d_t | d_h | d_w) & 1) ||
+        d_t + d_h + d_w != p->D)
+        return WF_ERR_INVALID_ARG;
+    p->rope.dt = d_t;
+    p->rope.dh = d_h;
+    p->rope.dw = d_w;
+    fill_rope_table(p->rope, p->theta);
+    return WF_OK;
+}
+
+int wf_plan_set_norm_eps(wf_plan_t p, double eps)
+{
+    if (p == nullptr || !(eps >= 0.0)) return WF_ERR_INVALID_ARG;
+    p->eps = eps;
+    return WF_OK;
+}
+
+int wf_plan_set_wait_limit(wf_plan_t p, unsigned long long cycles)
+{
+    if (p == nullptr) return WF_ERR_INVALID_ARG;
+    p->wait_limit = cycles == 0 ? kDefaultWaitLimit : cycles;
+    return WF_OK;
+}
+
+void wf_plan_destroy(wf_plan_t p)
+{
+    if (p == nullptr) return;
+    if (p->words != nullptr) {
+        int cur = -1;
+        const bool switch_dev = cudaGetDevice(&cur) == cudaSuccess && cur != p->device;
+        if (switch_dev) cudaSetDevice(p->device);
+        cudaFree(p->words);
+        if (switch_dev) cudaSetDevice(cur);
+    }
+    delete p;
+}
+
+size_t wf_cache_bytes(wf_plan_t p)
+{
+    if (p == nullptr) return 0;
+    return static_cast<size_t>(p->R) * p->L * p->H * p->D * 2;
+}
+
+double wf_useful_flops(wf_plan_t p, long round)
+{
+    if (p == nullptr || round < 0) return -1.0;
+    const int hv = wf::history_valid(round, p->Hh);
+    double chunks = 0.0;
+    for (int c = 0; c < p->W; ++c) chunks += hv + c + 1;
+    return 4.0 * p->H * p->D * static_cast<double>(p->L) * p->L * chunks;
+}
+
+int wf_qk_norm_rope_append(wf_plan_t p, long round, const void *q, const void *k, const void *v,
+                           const int32_t *pos_thw, const float *gamma_q, const float *gamma_k,
+                           void *q_out, void *k_cache, void *v_cache, void *stream)
+{
+    if (p == nullptr || round < 0) return WF_ERR_INVALID_ARG;
+    if (!q || !k || !v || !gamma_q || !gamma_k || !q_out || !k_cache || !v_cache)
+        return WF_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_out) ||
+        !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(gamma_q) || !aligned16(gamma_k))
+        return WF_ERR_INVALID_ARG;
+    if (pos_thw == nullptr && p->rope.F == 0) return WF_ERR_INVALID_ARG;
+    if (pos_thw != nullptr && (reinterpret_cast<uintptr_t>(pos_thw) & 3u)) return WF_ERR_INVALID_ARG;
+    if (pos_thw == nullptr &&
+        (round + p->W) > static_cast<long>(INT_MAX / p->rope.F))
+        return WF_ERR_INVALID_ARG;
+    if (int s = check_device(p)) return s;
+
+    wf::AppendParams a;
+    a.q = static_cast<const uint16_t *>(q);
+    a.k = static_cast<const uint16_t *>(k);
+    a.v = static_cast<const uint16_t *>(v);
+    a.pos = pos_thw;
+    a.gamma_q = gamma_q;
+    a.gamma_k = gamma_k;
+    a.q_out = static_cast<uint16_t *>(q_out);
+    a.k_cache = static_cast<uint16_t *>(k_cache);
+    a.v_cache = static_cast<uint16_t *>(v_cache);
+    a.round = round;
+    a.L = p->L;
+    a.W = p->W;
+    a.R = p->R;
+    a.H = p->H;
+    a.eps = static_cast<float>(p->eps);
+    a.rope = p->rope;
+    cudaError_t e = wf::launch_append(a, p->D, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? WF_OK : WF_ERR_CUDA;
+}
+
+int wf_chunk_causal_attn(wf_plan_t p, long round, const void *q_out, const void *k_cache,
+                         const void *v_cache, void *o, float *lse, void *stream)
+{
+    if (p == nullptr || round < 0) return WF_ERR_INVALID_ARG;
+    if (!q_out || !k_cache || !v_cache || !o) return WF_ERR_INVALID_ARG;
+    if (!aligned16(q_out) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+        (reinterpret_cast<uintptr_t>(lse) & 3u))
+        return WF_ERR_INVALID_ARG;
+    if (int s = check_device(p)) return s;
+
+    CUtensorMap mq, mk, mv;
+    if (!encode_map(&mq, q_out, p->D, p->H, p->L, p->L, p->W) ||
+        !encode_map(&mk, k_cache, p->D, p->H, p->L, p->L, p->R) ||
+        !encode_map(&mv, v_cache, p->D, p->H, p->L, p->L, p->R))
+        return WF_ERR_CUDA;
+
+    wf::AttnParams a;
+    a.round = round;
+    a.L = p->L;
+    a.W = p->W;
+    a.R = p->R;
+    a.H = p->H;
+    a.T = p->L * p->W;
+    a.h_valid = wf::history_valid(round, p->Hh);
+    a.n_ktiles = (p->L + 127) / 128;
+    a.n_qpairs = (a.n_ktiles + 1) / 2;
+    a.n_units = p->H * p->W * a.n_qpairs;
+    a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(p->D)));
+    a.wait_limit = p->wait_limit;
+    a.o = static_cast<uint16_t *>(o);
+    a.lse = lse;
+    a.words = p->words;
+    const int grid = a.n_units < p->num_sms ? a.n_units : p->num_sms;
+    cudaError_t e = wf::launch_attn(mq, mk, mv, a, p->D, grid, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? WF_OK : WF_ERR_CUDA;
+}
+
+int wf_sync_status(wf_plan_t p, void *stream)
+{
+    if (p == nullptr) return WF_ERR_INVALID_ARG;
+    if (int s = check_device(p)) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    wf::DeviceWords host;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return WF_ERR_CUDA;
+    if (cudaMemcpyAsync(&host, p->words, 2 * sizeof(uint32_t), cudaMemcpyDeviceToHost, st) !=
+            cudaSuccess ||
+        cudaMemsetAsync(p->words, 0, 2 * sizeof(uint32_t), st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return WF_ERR_CUDA;
+    if (host.status & wf::kStatusTimeout) return WF_ERR_TIMEOUT;
+    return WF_OK;
+}
+
+int wf_plan_debug_ranges(wf_plan_t p, long round, int32_t *out, int cap)
+{
+    if (p == nullptr || round < 0 || cap < 0 || (cap > 0 && out == nullptr)) return -1;
+    const int hv = wf::history_valid(round, p->Hh);
+    int n = 0;
+    for (int c = 0; c < p->W; ++c)
+        for (int b = 0; b <= hv + c; ++b, ++n) {
+            if (n >= cap) continue;
+            const long id = wf::visible_chunk_id(round, hv, b);
+            out[4 * n + 0] = c;
+            out[4 * n + 1] = b;
+            out[4 * n + 2] = static_cast<int32_t>(id);
+            out[4 * n + 3] = wf::ring_slot(id, p->R);
+        }
+    return n;
+}
+
+const char *wf_status_string(int s)
+{
+    switch (s) {
+    case WF_OK: return "ok";
+    case WF_ERR_INVALID_ARG: return "invalid argument";
+    case WF_ERR_UNSUPPORTED: return "unsupported configuration";
+    case WF_ERR_CUDA: return "CUDA error";
+    case WF_ERR_TIMEOUT: return "device wait timed out";
+    case WF_ERR_NO_DEVICE: return "plan has no device state";
+    case WF_ERR_DEVICE: return "device is not sm_100";
+    default: return "unknown status";
+    }
+}
+
+}  // extern "C"

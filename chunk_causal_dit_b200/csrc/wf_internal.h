@@ -1,0 +1,96 @@
+// wf_internal.h -- plan structure, kernel parameter blocks and the ring/visibility
+// arithmetic shared by host code (wf_plan_debug_ranges, launch set-up) and the
+// kernels, so that what the debug dump reports is what the kernels execute.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#ifdef __CUDACC__
+#define WF_HD __host__ __device__ __forceinline__
+#else
+#define WF_HD inline
+#endif
+
+namespace wf {
+
+constexpr int kMaxHeadDim = 128;
+
+// Number of history chunks visible in round r: min(Hh, r) (rounds before the
+// pipeline is full see fewer).
+WF_HD int history_valid(long round, int n_hist)
+{
+    return round < static_cast<long>(n_hist) ? static_cast<int>(round) : n_hist;
+}
+
+// Non-negative modulo for ring slots.
+WF_HD int ring_slot(long chunk_id, int R)
+{
+    long s = chunk_id % R;
+    return static_cast<int>(s < 0 ? s + R : s);
+}
+
+// Absolute id of the b-th visible key chunk (b = 0 is the oldest) in round r.
+WF_HD long visible_chunk_id(long round, int h_valid, int b)
+{
+    return round - h_valid + b;
+}
+
+// Status bits written by kernels into the plan's device status word.
+enum : uint32_t {
+    kStatusTimeout = 1u,
+};
+
+// Device-resident words owned by a plan (one 256-byte allocation).
+struct DeviceWords {
+    uint32_t status;          // OR of kStatus* bits
+    uint32_t timeout_where;   // role/barrier code of the first timeout
+    uint32_t sched_counter;   // attention work-unit counter (reset before each launch)
+    uint32_t pad[61];
+};
+
+struct RopeParams {
+    int dt, dh, dw;           // channel widths of the t / h / w blocks
+    int F, gh, gw;            // chunk geometry for derived positions (F = 0: unset)
+    float omega[kMaxHeadDim / 2];   // per channel pair: theta^(-2i/d_axis)
+    int8_t axis[kMaxHeadDim / 2];   // per channel pair: 0 = t, 1 = h, 2 = w
+};
+
+struct AppendParams {
+    const uint16_t *q, *k, *v;
+    const int32_t *pos;       // [T,3] or nullptr (derive)
+    const float *gamma_q, *gamma_k;
+    uint16_t *q_out, *k_cache, *v_cache;
+    long round;
+    int L, W, R, H;
+    float eps;
+    RopeParams rope;
+};
+
+struct AttnParams {
+    long round;
+    int L, W, R, H, T;
+    int h_valid;
+    int n_qpairs;             // query tile pairs per chunk: ceil(ceil(L/128)/2)
+    int n_ktiles;             // key tiles per chunk: ceil(L/128)
+    int n_units;              // H * W * n_qpairs
+    float scale_log2;         // log2(e) / sqrt(D)
+    unsigned long long wait_limit;  // SM clock cycles
+    uint16_t *o;
+    float *lse;
+    DeviceWords *words;
+};
+
+}  // namespace wf
+
+struct wf_plan_s {
+    int L, W, Hh, H, D, R;
+    double theta;
+    double eps;
+    wf::RopeParams rope;
+    unsigned long long wait_limit;
+    int device;               // -1: no device state
+    int num_sms;
+    int cc_major, cc_minor;   // compute capability of `device`
+    wf::DeviceWords *words;   // device memory
+};

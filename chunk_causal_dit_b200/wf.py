@@ -1,0 +1,190 @@
+"""ctypes binding of libwf.so with the C ABI's names (argument marshalling only).
+
+Every step of the hot path runs in the library's CUDA kernels; this module only
+turns torch tensors (or raw integers) into pointers and status codes into
+exceptions.  Loading fails loudly if the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libwf.so")
+
+WF_OK = 0
+WF_ERR_INVALID_ARG = 1
+WF_ERR_UNSUPPORTED = 2
+WF_ERR_CUDA = 3
+WF_ERR_TIMEOUT = 4
+WF_ERR_NO_DEVICE = 5
+WF_ERR_DEVICE = 6
+
+# Every function include/wf.h declares: name -> (restype, argtypes)
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_L = ctypes.c_long
+SIGNATURES = {
+    "wf_plan": (_I, [_I, _I, _I, _I, _I, ctypes.POINTER(_P)]),
+    "wf_plan_set_rope": (_I, [_P, _I, _I, _I, ctypes.c_double]),
+    "wf_plan_set_rope_split": (_I, [_P, _I, _I, _I]),
+    "wf_plan_set_norm_eps": (_I, [_P, ctypes.c_double]),
+    "wf_plan_set_wait_limit": (_I, [_P, ctypes.c_ulonglong]),
+    "wf_plan_destroy": (None, [_P]),
+    "wf_cache_bytes": (ctypes.c_size_t, [_P]),
+    "wf_useful_flops": (ctypes.c_double, [_P, _L]),
+    "wf_qk_norm_rope_append": (_I, [_P, _L, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "wf_chunk_causal_attn": (_I, [_P, _L, _P, _P, _P, _P, _P, _P]),
+    "wf_sync_status": (_I, [_P, _P]),
+    "wf_plan_debug_ranges": (_I, [_P, _L, _P, _I]),
+    "wf_status_string": (ctypes.c_char_p, [_I]),
+}
+
+_lib = None
+
+
+class WFError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__("%s: %s (status %d)" % (what, status_string(status), status))
+
+
+def load() -> ctypes.CDLL:
+    """Load libwf.so (built in-tree by chunk_causal_dit_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError("libwf.so not built: run `python -m chunk_causal_dit_b200.build` "
+                              "(expected at %s)" % LIB_PATH)
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return load().wf_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != WF_OK:
+        raise WFError(status, what)
+
+
+def _ptr(x) -> Optional[int]:
+    """torch tensor / int / None -> raw pointer value."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        try:
+            import torch
+            if torch.cuda.is_available():
+                return torch.cuda.current_stream().cuda_stream
+        except Exception:
+            pass
+        return None
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+class Plan:
+    """Owns a wf_plan_t; mirrors wf_plan / wf_plan_set_* / wf_plan_destroy."""
+
+    def __init__(self, chunk_tokens: int, n_wave_chunks: int, n_hist_chunks: int, heads: int,
+                 head_dim: int):
+        self.L, self.W, self.Hh, self.H, self.D = (chunk_tokens, n_wave_chunks, n_hist_chunks,
+                                                   heads, head_dim)
+        self.R = n_hist_chunks + n_wave_chunks
+        self.T = chunk_tokens * n_wave_chunks
+        h = ctypes.c_void_p()
+        _check(load().wf_plan(chunk_tokens, n_wave_chunks, n_hist_chunks, heads, head_dim,
+                              ctypes.byref(h)), "wf_plan")
+        self.handle = h.value
+
+    def set_rope(self, frames_per_chunk: int, grid_h: int, grid_w: int, theta: float = 10000.0):
+        _check(load().wf_plan_set_rope(self.handle, frames_per_chunk, grid_h, grid_w, theta),
+               "wf_plan_set_rope")
+        return self
+
+    def set_rope_split(self, d_t: int, d_h: int, d_w: int):
+        _check(load().wf_plan_set_rope_split(self.handle, d_t, d_h, d_w), "wf_plan_set_rope_split")
+        return self
+
+    def set_norm_eps(self, eps: float):
+        _check(load().wf_plan_set_norm_eps(self.handle, eps), "wf_plan_set_norm_eps")
+        return self
+
+    def set_wait_limit(self, cycles: int):
+        _check(load().wf_plan_set_wait_limit(self.handle, cycles), "wf_plan_set_wait_limit")
+        return self
+
+    def destroy(self):
+        if self.handle:
+            load().wf_plan_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.destroy()
+
+
+def wf_plan(chunk_tokens, n_wave_chunks, n_hist_chunks, heads, head_dim) -> Plan:
+    return Plan(chunk_tokens, n_wave_chunks, n_hist_chunks, heads, head_dim)
+
+
+def wf_cache_bytes(plan: Plan) -> int:
+    return int(load().wf_cache_bytes(plan.handle))
+
+
+def wf_useful_flops(plan: Plan, round_: int) -> float:
+    return float(load().wf_useful_flops(plan.handle, round_))
+
+
+def wf_qk_norm_rope_append(plan: Plan, round_: int, q, k, v, pos_thw, gamma_q, gamma_k, q_out,
+                           k_cache, v_cache, stream=None) -> None:
+    _check(load().wf_qk_norm_rope_append(plan.handle, round_, _ptr(q), _ptr(k), _ptr(v),
+                                         _ptr(pos_thw), _ptr(gamma_q), _ptr(gamma_k),
+                                         _ptr(q_out), _ptr(k_cache), _ptr(v_cache),
+                                         _stream(stream)), "wf_qk_norm_rope_append")
+
+
+def wf_chunk_causal_attn(plan: Plan, round_: int, q_out, k_cache, v_cache, o, lse=None,
+                         stream=None) -> None:
+    _check(load().wf_chunk_causal_attn(plan.handle, round_, _ptr(q_out), _ptr(k_cache),
+                                       _ptr(v_cache), _ptr(o), _ptr(lse), _stream(stream)),
+           "wf_chunk_causal_attn")
+
+
+def wf_sync_status(plan: Plan, stream=None) -> int:
+    """Returns the status code (WF_OK or WF_ERR_TIMEOUT ...) without raising."""
+    return int(load().wf_sync_status(plan.handle, _stream(stream)))
+
+
+def wf_plan_debug_ranges(plan: Plan, round_: int):
+    """List of (wave chunk, logical index, absolute chunk id, ring slot) in visiting order."""
+    lib = load()
+    n = lib.wf_plan_debug_ranges(plan.handle, round_, None, 0)
+    if n < 0:
+        raise WFError(WF_ERR_INVALID_ARG, "wf_plan_debug_ranges")
+    buf = (ctypes.c_int32 * (4 * max(n, 1)))()
+    lib.wf_plan_debug_ranges(plan.handle, round_, buf, n)
+    return [tuple(buf[4 * i:4 * i + 4]) for i in range(n)]

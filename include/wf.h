@@ -1,0 +1,150 @@
+/*
+ * wf.h -- C ABI of libwf.so: the wave-round hot path of Wave Forcing on B200.
+ *
+ * Source of the operations: "Wave Forcing: Towards Speed-of-Light Streaming
+ * Video Generation" (abstract): one concurrent forward round ("wave") runs S
+ * chunks at staggered denoising steps plus one cache-refresh chunk; chunk-wise
+ * causal attention lets each chunk read earlier, cleaner chunks (including
+ * ones whose denoising is not finished) and the rolling history cache; Wave
+ * Parallelism delivers each layer's K/V early.  The airadar.tv summary
+ * ("usage") fixes the wave sizes (--rf-step 4 --wp-size 5, --rf-step 5
+ * --wp-size 6) and 3-latent-frame chunks.
+ *
+ * Notation.  L = tokens per chunk, W = chunks in the wave (denoising chunks +
+ * the refresh chunk, refresh chunk = wave chunk 0, the oldest), Hh = history
+ * chunks, H = heads, D = head_dim, T = W*L, R = Hh + W ring slots.  In round r
+ * wave chunk c is absolute chunk r + c; the history is the h = min(Hh, r)
+ * chunks r-h .. r-1.  Absolute chunk g lives in ring slot g mod R.
+ *
+ * Layouts (all row-major, bf16 = 16-bit bfloat16 bit patterns):
+ *   q, k, v, q_out, o     [T][H][D]  token-major, as a QKV projection emits
+ *   k_cache, v_cache      [R][L][H][D]
+ *   pos_thw               [T][3] int32 (t, h, w) or NULL (derived, see below)
+ *   gamma_q, gamma_k      [H][D] float32
+ *   lse                   [H][T] float32 natural-log sum-exp, or NULL
+ *
+ * Ownership.  The caller owns every buffer and stream.  The library owns the
+ * plan (host memory plus a few bytes of device memory on the device that was
+ * current at wf_plan, freed by wf_plan_destroy).  The two hot calls allocate
+ * nothing, never synchronise the host and use only the stream they are given
+ * (NULL = the legacy default stream).  They are asynchronous: errors raised on
+ * the device are reported by wf_sync_status.  Hot calls of one plan must not
+ * run concurrently on the GPU (the plan's device words are shared).
+ *
+ * Errors.  Every entry point returns a wf_status (0 = WF_OK) or a value that
+ * documents its own failure value.  Nothing aborts the process, nothing traps
+ * on the device; a device-side wait that runs past its limit ends the kernel
+ * with WF_ERR_TIMEOUT recorded in the plan.
+ */
+#ifndef WF_H_
+#define WF_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define WF_API __attribute__((visibility("default")))
+#else
+#define WF_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum wf_status {
+    WF_OK = 0,
+    WF_ERR_INVALID_ARG = 1,   /* a size, pointer or alignment check failed        */
+    WF_ERR_UNSUPPORTED = 2,   /* valid but not built (e.g. head_dim not 64/128)    */
+    WF_ERR_CUDA = 3,          /* a CUDA runtime/driver call or launch failed       */
+    WF_ERR_TIMEOUT = 4,       /* a bounded device wait expired (kernel stopped)    */
+    WF_ERR_NO_DEVICE = 5,     /* the plan has no device state (no GPU at wf_plan)  */
+    WF_ERR_DEVICE = 6         /* the device is not an sm_100 (B200-class) part     */
+} wf_status;
+
+typedef struct wf_plan_s *wf_plan_t;
+
+/* Build a plan for one layer's wave round.
+ * chunk_tokens L >= 1, n_wave_chunks W >= 1, n_hist_chunks Hh >= 0, heads H >= 1,
+ * head_dim D in {64, 128}; T*H*D must fit in 2^31 elements per tensor.
+ * Host work only, plus a 256-byte device allocation (status word and the
+ * attention scheduler's counter) on the current device.  If no CUDA device is
+ * present the plan is still created for the host-side queries and the hot
+ * calls return WF_ERR_NO_DEVICE.  RoPE defaults: no grid set (pos_thw must be
+ * passed), split dt = D - 4*(D/6), dh = dw = 2*(D/6), theta = 10000;
+ * RMSNorm eps = 1e-6.  *out is NULL on failure. */
+WF_API int wf_plan(int chunk_tokens, int n_wave_chunks, int n_hist_chunks, int heads,
+            int head_dim, wf_plan_t *out);
+
+/* Latent geometry of a chunk for derived positions: L must equal
+ * frames_per_chunk * grid_h * grid_w.  Token n = c*L + f*grid_h*grid_w + y*grid_w + x
+ * of round r gets (t, h, w) = ((r + c)*frames_per_chunk + f, y, x).  theta > 0. */
+WF_API int wf_plan_set_rope(wf_plan_t plan, int frames_per_chunk, int grid_h, int grid_w,
+                     double theta);
+
+/* Channel widths of the t/h/w RoPE blocks (each even, sum = D). */
+WF_API int wf_plan_set_rope_split(wf_plan_t plan, int d_t, int d_h, int d_w);
+
+/* RMSNorm epsilon (>= 0). */
+WF_API int wf_plan_set_norm_eps(wf_plan_t plan, double eps);
+
+/* Device-wait limit in SM clock cycles for the attention kernel (0 = default,
+ * about two seconds).  Exposed so that tests can make a wait expire quickly. */
+WF_API int wf_plan_set_wait_limit(wf_plan_t plan, unsigned long long cycles);
+
+WF_API void wf_plan_destroy(wf_plan_t plan);
+
+/* Bytes of ONE ring (K or V): R * L * H * D * 2.  0 for a NULL plan. */
+WF_API size_t wf_cache_bytes(wf_plan_t plan);
+
+/* Useful attention FLOPs of round r: 4*H*D*L^2 * sum_c (min(Hh, r) + c + 1),
+ * i.e. QK^T and PV over visible, unpadded pairs.  -1 for a NULL plan. */
+WF_API double wf_useful_flops(wf_plan_t plan, long round);
+
+/* Fused per-head RMSNorm(q, k) * gamma, 3D RoPE, and ring append.
+ * For every wave token n (chunk c = n / L) and head h:
+ *   q_out[n,h] = bf16(RoPE(pos[n], RMSNorm(q[n,h]) * gamma_q[h]))
+ *   k_cache[(r+c) mod R, n mod L, h] = bf16(RoPE(pos[n], RMSNorm(k[n,h]) * gamma_k[h]))
+ *   v_cache[(r+c) mod R, n mod L, h] = v[n,h]          (bit-exact copy)
+ * fp32 arithmetic, one round-to-nearest-even to bf16.  round >= 0.  All
+ * pointers are device pointers, 16-byte aligned; pos_thw may be NULL when
+ * wf_plan_set_rope set the geometry.  q_out may alias q; nothing else may
+ * overlap.  One kernel launch on `stream` (a cudaStream_t). */
+WF_API int wf_qk_norm_rope_append(wf_plan_t plan, long round,
+                           const void *q, const void *k, const void *v,
+                           const int32_t *pos_thw,
+                           const float *gamma_q, const float *gamma_k,
+                           void *q_out, void *k_cache, void *v_cache,
+                           void *stream);
+
+/* Chunk-causal attention of round r.  For query token n of wave chunk c, head h:
+ *   O[n,h] = softmax_j(q_out[n,h] . K_j / sqrt(D)) V_j
+ * over every token j of the min(Hh, r) history chunks and of wave chunks 0..c
+ * (bidirectional inside a chunk), read from the ring slots written by
+ * wf_qk_norm_rope_append.  bf16 tensor-core products, fp32 accumulation and
+ * softmax, one rounding of O to bf16.  lse (optional) gets the natural-log
+ * sum-exp per (h, n).  Device pointers, 16-byte aligned; o must not overlap the
+ * inputs.  One persistent kernel launch (plus a 4-byte memset of the scheduler
+ * counter) on `stream`. */
+WF_API int wf_chunk_causal_attn(wf_plan_t plan, long round,
+                         const void *q_out, const void *k_cache, const void *v_cache,
+                         void *o, float *lse, void *stream);
+
+/* Wait for `stream`, then read and clear the plan's device status word.
+ * Returns WF_OK, WF_ERR_TIMEOUT (a bounded device wait expired) or WF_ERR_CUDA. */
+WF_API int wf_sync_status(wf_plan_t plan, void *stream);
+
+/* The key chunks the attention kernel visits in round r, in visiting order:
+ * for each wave chunk c, for each visible chunk (oldest first), the quadruple
+ * (c, logical index b, absolute chunk id, ring slot).  Writes at most cap
+ * quadruples (4*cap int32) and returns the number needed, or -1 on bad input.
+ * The kernel computes slots with the same function. */
+WF_API int wf_plan_debug_ranges(wf_plan_t plan, long round, int32_t *out, int cap);
+
+WF_API const char *wf_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WF_H_ */

@@ -1,0 +1,139 @@
+"""C-ABI checks that need no GPU: symbols, argument validation, host-side logic.
+
+The ring/visibility arithmetic that wf_plan_debug_ranges reports is the same
+function the attention kernel calls; here it is checked against the oracle's
+cache model, which keys chunks by absolute id and has no ring.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from chunk_causal_dit_b200 import build as wf_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def wf():
+    wf_build.build()
+    from chunk_causal_dit_b200 import wf as mod
+    mod.load()
+    return mod
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "wf.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(wf_[a-z_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol(wf):
+    names = header_functions()
+    assert len(names) >= 13
+    lib = ctypes.CDLL(wf.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(wf.SIGNATURES), "binding and header disagree"
+
+
+def test_plan_argument_validation(wf):
+    lib = wf.load()
+    h = ctypes.c_void_p()
+    bad = [(0, 5, 2, 12, 128), (4680, 0, 2, 12, 128), (4680, 5, -1, 12, 128),
+           (4680, 5, 2, 0, 128)]
+    for args in bad:
+        assert lib.wf_plan(*args, ctypes.byref(h)) == wf.WF_ERR_INVALID_ARG
+        assert h.value is None
+    assert lib.wf_plan(4680, 5, 2, 12, 96, ctypes.byref(h)) == wf.WF_ERR_UNSUPPORTED
+    # too large for 32-bit element indexing of one [T,H,D] tensor
+    assert lib.wf_plan(1 << 20, 64, 0, 64, 128, ctypes.byref(h)) == wf.WF_ERR_INVALID_ARG
+    assert lib.wf_plan(4680, 5, 2, 12, 128, None) == wf.WF_ERR_INVALID_ARG
+
+
+def test_plan_setters_validate(wf):
+    p = wf.Plan(4680, 5, 2, 12, 128)
+    with pytest.raises(wf.WFError):
+        p.set_rope(3, 30, 51)              # 3*30*51 != 4680
+    p.set_rope(3, 30, 52)
+    with pytest.raises(wf.WFError):
+        p.set_rope_split(44, 42, 40)       # sum != D
+    with pytest.raises(wf.WFError):
+        p.set_rope_split(43, 43, 42)       # odd widths
+    p.set_rope_split(44, 42, 42)
+    with pytest.raises(wf.WFError):
+        p.set_norm_eps(-1.0)
+    p.set_norm_eps(1e-5)
+    p.destroy()
+
+
+@pytest.mark.parametrize("L,W,Hh,H,D", [(32, 3, 0, 2, 64), (4680, 5, 2, 12, 128),
+                                        (4680, 6, 3, 12, 128), (4680, 5, 3, 40, 128),
+                                        (100, 4, 7, 3, 64)])
+def test_useful_flops_and_cache_bytes(wf, L, W, Hh, H, D):
+    p = wf.Plan(L, W, Hh, H, D)
+    for r in (0, 1, 2, 3, 10):
+        assert wf.wf_useful_flops(p, r) == oracle.useful_flops(L, W, Hh, H, D, r)
+    assert wf.wf_cache_bytes(p) == (Hh + W) * L * H * D * 2
+    p.destroy()
+
+
+def test_useful_flops_headline_value(wf):
+    # 12 heads x 128, 4680-token chunks, 5-chunk wave, 2 history chunks: 3.364 TFLOP
+    p = wf.Plan(4680, 5, 2, 12, 128)
+    assert abs(wf.wf_useful_flops(p, 2) - 3.3644e12) < 0.001e12
+    p.destroy()
+
+
+@pytest.mark.parametrize("W,Hh", [(3, 0), (5, 2), (6, 3), (2, 5)])
+def test_debug_ranges_match_oracle_cache_model(wf, W, Hh):
+    L, H = 4, 1
+    p = wf.Plan(L, W, Hh, H, 64)
+    R = W + Hh
+    cache = oracle.OracleCache(L)
+    for r in range(0, 2 * R + 3):
+        got = wf.wf_plan_debug_ranges(p, r)
+        # oracle: ids visible to wave chunk c are the round's history then chunks r..r+c
+        for i in range(r - min(Hh, r), r + W):
+            cache.put(i, np.zeros((L, H, 64), np.uint16), np.zeros((L, H, 64), np.uint16))
+        _, _, ids = cache.round_keys(r, W, Hh)
+        hv = len(ids) - W
+        want = []
+        for c in range(W):
+            for b, cid in enumerate(ids[:hv + c + 1]):
+                want.append((c, b, int(cid), int(cid) % R))
+        assert got == want
+        # within one round every visible chunk has its own slot
+        slots = {s for (_, _, _, s) in got}
+        assert len(slots) == len(ids)
+
+
+def test_hot_calls_without_device(wf):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("device present")
+    p = wf.Plan(32, 3, 0, 2, 64)
+    lib = wf.load()
+    fake = 1 << 20   # never dereferenced: the call fails before any launch
+    assert lib.wf_chunk_causal_attn(p.handle, 0, fake, fake, fake, fake, None, None) == \
+        wf.WF_ERR_NO_DEVICE
+    assert lib.wf_qk_norm_rope_append(p.handle, 0, fake, fake, fake, None, fake, fake, fake,
+                                      fake, fake, None) == wf.WF_ERR_INVALID_ARG  # no geometry
+    p.set_rope(2, 4, 4)
+    assert lib.wf_qk_norm_rope_append(p.handle, 0, fake, fake, fake, None, fake, fake, fake,
+                                      fake, fake, None) == wf.WF_ERR_NO_DEVICE
+    # misaligned pointers are rejected before the device check
+    assert lib.wf_chunk_causal_attn(p.handle, 0, fake + 2, fake, fake, fake, None, None) == \
+        wf.WF_ERR_INVALID_ARG
+    assert lib.wf_chunk_causal_attn(p.handle, -1, fake, fake, fake, fake, None, None) == \
+        wf.WF_ERR_INVALID_ARG
+    p.destroy()
+
+
+def test_status_strings(wf):
+    assert wf.status_string(0) == "ok"
+    assert "timed out" in wf.status_string(wf.WF_ERR_TIMEOUT)
+    assert wf.status_string(999) == "unknown status"

@@ -1,0 +1,219 @@
+"""GPU parity of wf_chunk_causal_attn against the fp64 oracle.
+
+Bars (unit-scale data, fp32 accumulation, bf16 output): max abs error <= 1e-2
+and mean abs error <= 1e-3 per case; lse within 1e-3.  Chunk visibility and
+ring indexing are exact: perturbing a later chunk leaves earlier chunks'
+outputs bit-identical, and rounds that wrap the ring match the oracle's
+absolute-id cache model.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from chunk_causal_dit_b200 import build as wf_build
+from chunk_causal_dit_b200 import inputs as wi
+from tests.wfcase import (assert_attention_close, assert_attention_within_rounding,
+                          rand_bf16, sample_rows)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def wf():
+    wf_build.build()
+    from chunk_causal_dit_b200 import wf as mod
+    return mod
+
+
+def place_round(L, W, Hh, H, D, round_, seed):
+    """Random q_out and a ring whose slot (g mod R) holds absolute chunk g."""
+    R = Hh + W
+    q = rand_bf16((W * L, H, D), seed)
+    kc = rand_bf16((R, L, H, D), seed + 1)
+    vc = rand_bf16((R, L, H, D), seed + 2)
+    return q, kc, vc
+
+
+def oracle_cache_from_ring(kc, vc, round_, W, Hh):
+    """The oracle's absolute-id view of a ring laid out by the header contract."""
+    L = kc.shape[1]
+    R = kc.shape[0]
+    cache = oracle.OracleCache(L)
+    kb, vb = wi.bits(kc.cpu()), wi.bits(vc.cpu())
+    for g in range(round_ - min(Hh, round_), round_ + W):
+        cache.put(g, kb[g % R], vb[g % R])
+    return cache
+
+
+def run_attn(wf, plan, round_, q, kc, vc, with_lse=True):
+    T, H, D = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((H, T), dtype=torch.float32, device=q.device) if with_lse else None
+    wf.wf_chunk_causal_attn(plan, round_, q, kc, vc, o, lse)
+    torch.cuda.synchronize()
+    assert wf.wf_sync_status(plan) == wf.WF_OK
+    return o, lse
+
+
+SHAPES = [
+    # L, W, Hh, H, D, round
+    (300, 4, 2, 3, 128, 5),     # ragged chunk: 2 full tiles + 44 rows
+    (200, 3, 1, 2, 64, 7),      # head_dim 64, ragged
+    (128, 2, 0, 1, 128, 0),     # exactly one tile, no history
+    (129, 3, 3, 2, 128, 1),     # one row past a tile; pipeline filling (1 of 3 history)
+    (1, 3, 1, 2, 64, 4),        # one token per chunk
+    (513, 2, 2, 1, 128, 9),     # 5 tiles, last with 1 row; odd number of query tiles
+    (32, 3, 0, 2, 64, 0),       # the tiny wave shape
+]
+
+
+@pytest.mark.parametrize("L,W,Hh,H,D,r", SHAPES)
+def test_attention_all_rows(wf, L, W, Hh, H, D, r):
+    q, kc, vc = place_round(L, W, Hh, H, D, r, seed=L + W + D)
+    plan = wf.Plan(L, W, Hh, H, D)
+    o, lse = run_attn(wf, plan, r, q, kc, vc)
+    cache = oracle_cache_from_ring(kc, vc, r, W, Hh)
+    T = W * L
+    rows = np.repeat(np.arange(T), H)
+    heads = np.tile(np.arange(H), T)
+    o_ref, lse_ref = oracle.round_attention(cache, r, W, Hh, wi.bits(q.cpu()), rows, heads)
+    o_gpu = o.float().cpu().numpy().reshape(T * H, D)
+    what = "O L=%d W=%d Hh=%d D=%d r=%d" % (L, W, Hh, D, r)
+    if L * (min(Hh, r) + 1) >= 32:
+        assert_attention_close(o_gpu, o_ref, what)
+    else:   # a handful of visible keys per row: the elementwise rounding bound
+        v_absmax = float(vc.float().abs().max())
+        assert_attention_within_rounding(o_gpu, o_ref, v_absmax, what)
+    lse_gpu = lse.cpu().numpy().T.reshape(-1)
+    assert np.max(np.abs(lse_gpu - lse_ref)) <= 1e-3
+    plan.destroy()
+
+
+def test_causality_perturbation_bit_identical(wf):
+    L, W, Hh, H, D, r = 200, 4, 2, 2, 128, 6
+    q, kc, vc = place_round(L, W, Hh, H, D, r, seed=5)
+    plan = wf.Plan(L, W, Hh, H, D)
+    base, _ = run_attn(wf, plan, r, q, kc, vc)
+    R = W + Hh
+    for j in range(W):
+        kc2, vc2 = kc.clone(), vc.clone()
+        slot = (r + j) % R
+        kc2[slot] = rand_bf16((L, H, D), 100 + j)
+        vc2[slot] = rand_bf16((L, H, D), 200 + j)
+        pert, _ = run_attn(wf, plan, r, q, kc2, vc2)
+        assert torch.equal(pert[:j * L].view(torch.int16), base[:j * L].view(torch.int16))
+        assert not torch.equal(pert[j * L:], base[j * L:])
+    plan.destroy()
+
+
+def test_repeat_runs_bit_identical(wf):
+    L, W, Hh, H, D, r = 4680 // 4, 5, 2, 4, 128, 2
+    q, kc, vc = place_round(L, W, Hh, H, D, r, seed=9)
+    plan = wf.Plan(L, W, Hh, H, D)
+    first, lse0 = run_attn(wf, plan, r, q, kc, vc)
+    for _ in range(5):
+        again, lse1 = run_attn(wf, plan, r, q, kc, vc)
+        assert torch.equal(again.view(torch.int16), first.view(torch.int16))
+        assert torch.equal(lse1, lse0)
+    plan.destroy()
+
+
+def test_ring_over_rounds_end_to_end(wf):
+    # append + attention for rounds 0 .. 2R+1 against the oracle's absolute-id cache
+    w = wi.Workload("ring", H=2, D=64, F=1, gh=5, gw=8, n_wave=3, n_hist=2)
+    dev = "cuda"
+    plan = wf.Plan(w.L, w.n_wave, w.n_hist, w.H, w.D).set_rope(w.F, w.gh, w.gw)
+    kc = torch.zeros((w.R, w.L, w.H, w.D), dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros_like(kc)
+    cache = oracle.OracleCache(w.L)
+    rows = np.repeat(np.arange(w.T), w.H)
+    heads = np.tile(np.arange(w.H), w.T)
+    for r in range(2 * w.R + 2):
+        x = wi.wave_inputs(w, seed=0, salt=r)
+        q_out = torch.empty((w.T, w.H, w.D), dtype=torch.bfloat16, device=dev)
+        o = torch.empty_like(q_out)
+        wf.wf_qk_norm_rope_append(plan, r, x.q.to(dev), x.k.to(dev), x.v.to(dev), None,
+                                  x.gamma_q.to(dev), x.gamma_k.to(dev), q_out, kc, vc)
+        wf.wf_chunk_causal_attn(plan, r, q_out, kc, vc, o, None)
+        torch.cuda.synchronize()
+        assert wf.wf_sync_status(plan) == wf.WF_OK
+        pos = oracle.positions(r, w.n_wave, w.F, w.gh, w.gw)
+        qo, ko, vo = oracle.append(wi.bits(x.q), wi.bits(x.k), wi.bits(x.v), pos,
+                                   x.gamma_q.numpy(), x.gamma_k.numpy())
+        cache.put_wave(r, ko, vo)
+        o_ref, _ = oracle.round_attention(cache, r, w.n_wave, w.n_hist, qo, rows, heads)
+        assert_attention_close(o.float().cpu().numpy().reshape(-1, w.D), o_ref, "round %d" % r)
+    plan.destroy()
+
+
+def test_tiny_wave_end_to_end_and_isolated(wf):
+    w = wi.WORKLOADS["tiny"]
+    dev = "cuda"
+    x = wi.wave_inputs(w, seed=0)
+    plan = wf.Plan(w.L, w.n_wave, w.n_hist, w.H, w.D).set_rope(w.F, w.gh, w.gw)
+    q_out = torch.empty((w.T, w.H, w.D), dtype=torch.bfloat16, device=dev)
+    kc = torch.zeros((w.R, w.L, w.H, w.D), dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros_like(kc)
+    o = torch.empty_like(q_out)
+    wf.wf_qk_norm_rope_append(plan, 0, x.q.to(dev), x.k.to(dev), x.v.to(dev), None,
+                              x.gamma_q.to(dev), x.gamma_k.to(dev), q_out, kc, vc)
+    wf.wf_chunk_causal_attn(plan, 0, q_out, kc, vc, o, None)
+    torch.cuda.synchronize()
+    rows = np.repeat(np.arange(w.T), w.H)
+    heads = np.tile(np.arange(w.H), w.T)
+    # isolated: the oracle attends over the GPU's own q_out / K' / V
+    cache = oracle_cache_from_ring(kc, vc, 0, w.n_wave, w.n_hist)
+    o_iso, _ = oracle.round_attention(cache, 0, w.n_wave, w.n_hist, wi.bits(q_out.cpu()),
+                                      rows, heads)
+    got = o.float().cpu().numpy().reshape(-1, w.D)
+    assert_attention_close(got, o_iso, "tiny isolated")
+    # end to end: the oracle's own append feeds its attention
+    pos = oracle.positions(0, w.n_wave, w.F, w.gh, w.gw)
+    qo, ko, vo = oracle.append(wi.bits(x.q), wi.bits(x.k), wi.bits(x.v), pos,
+                               x.gamma_q.numpy(), x.gamma_k.numpy())
+    cache2 = oracle.OracleCache(w.L)
+    cache2.put_wave(0, ko, vo)
+    o_e2e, _ = oracle.round_attention(cache2, 0, w.n_wave, w.n_hist, qo, rows, heads)
+    assert_attention_close(got, o_e2e, "tiny end to end")
+    plan.destroy()
+
+
+@pytest.mark.parametrize("name,head_sel", [("wan13b_4step", None), ("wan13b_5step", [0, 5, 11]),
+                                           ("wan14b_4step", [0, 1, 22, 39])])
+def test_full_size_sampled(wf, name, head_sel):
+    """Full-size round r = n_hist (steady state), the launch the benchmark times;
+    checked on rows at chunk and tile boundaries plus random rows."""
+    w = wi.WORKLOADS[name]
+    dev = "cuda"
+    r = w.n_hist
+    x = wi.wave_inputs(w, seed=0)
+    hk, hv = wi.history_prefill(w, seed=0)
+    plan = wf.Plan(w.L, w.n_wave, w.n_hist, w.H, w.D).set_rope(w.F, w.gh, w.gw)
+    kc = torch.empty((w.R, w.L, w.H, w.D), dtype=torch.bfloat16, device=dev)
+    vc = torch.empty_like(kc)
+    for j in range(w.n_hist):                 # history chunk ids 0 .. n_hist-1
+        kc[j % w.R] = hk[j].to(dev)
+        vc[j % w.R] = hv[j].to(dev)
+    q_out = torch.empty((w.T, w.H, w.D), dtype=torch.bfloat16, device=dev)
+    o = torch.empty_like(q_out)
+    lse = torch.empty((w.H, w.T), dtype=torch.float32, device=dev)
+    wf.wf_qk_norm_rope_append(plan, r, x.q.to(dev), x.k.to(dev), x.v.to(dev), None,
+                              x.gamma_q.to(dev), x.gamma_k.to(dev), q_out, kc, vc)
+    wf.wf_chunk_causal_attn(plan, r, q_out, kc, vc, o, lse)
+    torch.cuda.synchronize()
+    assert wf.wf_sync_status(plan) == wf.WF_OK
+    cache = oracle_cache_from_ring(kc, vc, r, w.n_wave, w.n_hist)
+    sel = sample_rows(w.L, w.n_wave, 48, seed=1)
+    hs = list(range(w.H)) if head_sel is None else head_sel
+    rows = np.repeat(sel, len(hs))
+    heads = np.tile(hs, len(sel))
+    o_ref, lse_ref = oracle.round_attention(cache, r, w.n_wave, w.n_hist,
+                                            wi.bits(q_out.cpu()), rows, heads)
+    o_all = o.float().cpu().numpy()
+    got = o_all[rows, heads]
+    assert_attention_close(got, o_ref, name)
+    lse_all = lse.cpu().numpy()
+    assert np.max(np.abs(lse_all[heads, rows] - lse_ref)) <= 1e-3
+    assert np.isfinite(o_all).all()
+    plan.destroy()
