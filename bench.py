@@ -151,13 +151,19 @@ def barrier(dist, device=None):
             dist.barrier()
 
 
-def allreduce_max(dist, value, device):
+def allreduce_max(dist, value, device=None):
+    """Max of a per-rank scalar over all ranks (host-side timing reduction only)."""
     if dist is None:
         return value
     import torch
     t = torch.tensor([value], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_tflops(world, flops_per_rank_step, ms_step_max):
+    """Whole-job useful TFLOP/s: every rank's work over the slowest rank's time."""
+    return world * flops_per_rank_step / (ms_step_max * 1e-3) / 1e12
 
 
 # ------------------------------------------------------------------ ours --
@@ -206,7 +212,7 @@ def run_ours(args, rank, world, local):
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(local) if rank == 0 or True else None
+    clocks = ClockSampler(local)
     time.sleep(0.3)
     barrier(dist, dev)
     torch.cuda.synchronize(dev)
@@ -273,7 +279,7 @@ def run_ours(args, rank, world, local):
 
     peak_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     attn_tflops = flops_step / (attn_ms * 1e-3) / 1e12
-    value = world * flops_step / (ms_step * 1e-3) / 1e12
+    value = aggregate_tflops(world, flops_step, ms_step)
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     append_gbs = append_bytes / (append_ms * 1e-3) / 1e9
     line = {
@@ -322,7 +328,7 @@ def run_ours(args, rank, world, local):
             "bytes_per_launch": append_bytes,
         },
         "e2e": {
-            "value": round(world * flops_step / (e2e_ms * 1e-3) / 1e12, 3),
+            "value": round(aggregate_tflops(world, flops_step, e2e_ms), 3),
             "unit": "TFLOP/s",
             "ms_per_step": round(e2e_ms, 4),
             "h2d_bytes_per_step": 3 * tensor_bytes,

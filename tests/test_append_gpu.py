@@ -1,8 +1,10 @@
 """GPU parity of wf_qk_norm_rope_append against the fp64 oracle.
 
 Bar: q_out and K' equal the oracle's round-to-nearest-even bf16 or differ by
-one bf16 ulp (fp32 arithmetic on the GPU vs fp64 in the oracle); V and the ring
-slot of every chunk are bit-exact; slots outside the wave are untouched.
+one bf16 ulp, plus the fp32 rounding error of the GPU's rotation (2^-20 times
+the pair's length, which matters only where the rotation nearly cancels); V
+and the ring slot of every chunk are bit-exact; slots outside the wave are
+untouched.
 """
 import numpy as np
 import pytest
@@ -42,22 +44,22 @@ def run_append(wf, w, round_, seed=0, explicit_pos=False):
     torch.cuda.synchronize()
     assert wf.wf_sync_status(plan) == wf.WF_OK
     ref = oracle.append(wi.bits(x.q), wi.bits(x.k), wi.bits(x.v), pos_np, x.gamma_q.numpy(),
-                        x.gamma_k.numpy())
+                        x.gamma_k.numpy(), want_f64=True)
     out = (wi.bits(q_out.cpu()), wi.bits(kc.cpu()), wi.bits(vc.cpu()))
     plan.destroy()
     return x, ref, out
 
 
 def check_append(w, round_, ref, out):
-    qo_ref, ko_ref, vo_ref = ref
+    qo_ref, ko_ref, vo_ref, q64, k64 = ref
     qo, kc, vc = out
-    frac_q = assert_within_one_ulp(qo, qo_ref, "q_out")
+    frac_q = assert_within_one_ulp(qo, qo_ref, "q_out", q64)
     written = set()
     for c in range(w.n_wave):
         slot = (round_ + c) % w.R
         written.add(slot)
         sl = slice(c * w.L, (c + 1) * w.L)
-        assert_within_one_ulp(kc[slot], ko_ref[sl], "K' chunk %d" % c)
+        assert_within_one_ulp(kc[slot], ko_ref[sl], "K' chunk %d" % c, k64[sl])
         assert np.array_equal(vc[slot], vo_ref[sl]), "V chunk %d not bit-exact" % c
     for s in range(w.R):
         if s not in written:
