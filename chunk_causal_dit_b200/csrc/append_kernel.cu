@@ -5,10 +5,16 @@
 // every wave chunk's K/V into the ring-buffer history cache in the same pass
 // that normalises and rotates Q/K, so the attention kernel finds K/V in place.
 //
-// Memory-bound: 12*T*H*D bytes per call (read q, k, v; write q', K', V).  Each
-// thread owns 8 consecutive channels (one 16-byte vector per tensor) of one
-// (token, head) row; the D/8 threads of a row reduce the sum of squares with
-// shuffles.  RoPE pairs (2i, 2i+1) never straddle threads.
+// Memory-bound: 12*T*H*D bytes per call (read q, k, v; write q', K', V).
+// A block covers kTokens consecutive tokens for a group of heads.  Thread
+// (h, part) owns channels [8*part, 8*part + 8) of head h -- one 16-byte vector
+// per tensor -- and issues the loads of all kTokens tokens before computing.
+// The D/8 threads of a row reduce the sum of squares with shuffles; RoPE pairs
+// (2i, 2i+1) never straddle threads.  The rotation angles depend on the token
+// only, so each block computes them once per token in a prologue: the angle
+// pos * omega in fp64, reduced to [-pi, pi] in fp64, then fp32 sincos -- so the
+// fp32 error of the rotation stays a few ulps of the pair's length at any
+// position.
 #include <cuda_bf16.h>
 
 #include "sm100.cuh"
@@ -17,6 +23,9 @@
 namespace wf {
 
 namespace {
+
+constexpr int kTokens = 4;         // tokens per block
+constexpr int kMaxThreads = 512;   // threads per block (head groups split larger H)
 
 __device__ __forceinline__ void unpack8(const uint4 &u, float (&x)[8])
 {
@@ -39,109 +48,138 @@ __device__ __forceinline__ uint4 pack8(const float (&y)[8])
 }
 
 template <int D>
-__global__ void __launch_bounds__(256) qk_norm_rope_append_kernel(const AppendParams p)
+__global__ void __launch_bounds__(kMaxThreads) qk_norm_rope_append_kernel(const AppendParams p)
 {
-    constexpr int TPR = D / 8;   // threads per (token, head) row
-    __shared__ float s_omega[D / 2];
-    __shared__ int s_axis[D / 2];
-    for (int i = threadIdx.x; i < D / 2; i += blockDim.x) {
-        s_omega[i] = p.rope.omega[i];
-        s_axis[i] = p.rope.axis[i];
+    constexpr int TPR = D / 8;           // threads per (token, head) row
+    constexpr int NP = D / 2;            // RoPE pairs
+    __shared__ float2 s_cs[kTokens][NP];   // (cos, sin) per token and pair
+    __shared__ long s_off[kTokens];        // element offset of the token's row in the ring
+
+    const long T = static_cast<long>(p.W) * p.L;
+    const long n0 = static_cast<long>(blockIdx.x) * kTokens;
+
+    // ---- prologue: angles and ring rows of the block's tokens ----
+    for (int i = threadIdx.x; i < kTokens * NP; i += blockDim.x) {
+        const int tl = i / NP, pr = i - tl * NP;
+        const long n = n0 + tl;
+        if (n >= T) continue;
+        const int c = static_cast<int>(n / p.L);
+        const int ic = static_cast<int>(n - static_cast<long>(c) * p.L);
+        const int ax = p.rope.axis[pr];
+        long pos;
+        if (p.pos != nullptr) {
+            pos = __ldg(p.pos + 3 * n + ax);
+        } else {
+            const int hw = p.rope.gh * p.rope.gw;
+            const int f = ic / hw;
+            const int rem = ic - f * hw;
+            const int y = rem / p.rope.gw;
+            pos = ax == 0 ? (p.round + c) * p.rope.F + f : (ax == 1 ? y : rem - y * p.rope.gw);
+        }
+        const double ang = static_cast<double>(pos) * p.rope.omega[pr];
+        const double k = rint(ang * 0.15915494309189535);   // 1 / (2 pi)
+        const float red = static_cast<float>(fma(-k, 6.283185307179586, ang));
+        float sn, cs;
+        sincosf(red, &sn, &cs);
+        s_cs[tl][pr] = make_float2(cs, sn);
+        if (pr == 0) {
+            const int slot = ring_slot(p.round + c, p.R);
+            s_off[tl] = (static_cast<long>(slot) * p.L + ic) * p.H * D;
+        }
     }
     __syncthreads();
 
-    const long items = static_cast<long>(p.W) * p.L * p.H * TPR;
-    const long it = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
-    const unsigned mask = __ballot_sync(0xFFFFFFFFu, it < items);
-    if (it >= items) return;
+    const int hl = threadIdx.x / TPR;
+    const int part = threadIdx.x - hl * TPR;
+    const int h = blockIdx.y * p.heads_per_block + hl;
+    // the block is rounded up to whole warps; lanes past the group are idle
+    const bool active = hl < p.heads_per_block && h < p.H;
+    const int hh = active ? h : 0;       // inactive lanes still join the shuffles
 
-    const long row = it / TPR;                 // (token, head) row
-    const int part = static_cast<int>(it % TPR);
-    const long n = row / p.H;                  // wave token
-    const int h = static_cast<int>(row - n * p.H);
-    const int c = static_cast<int>(n / p.L);   // wave chunk
-    const int i = static_cast<int>(n - static_cast<long>(c) * p.L);
-
-    const long off = row * D + part * 8;
-    const uint4 uq = __ldcs(reinterpret_cast<const uint4 *>(p.q + off));
-    const uint4 uk = __ldcs(reinterpret_cast<const uint4 *>(p.k + off));
-    const uint4 uv = __ldcs(reinterpret_cast<const uint4 *>(p.v + off));
-
-    int pos[3];
-    if (p.pos != nullptr) {
-        pos[0] = __ldg(p.pos + 3 * n + 0);
-        pos[1] = __ldg(p.pos + 3 * n + 1);
-        pos[2] = __ldg(p.pos + 3 * n + 2);
-    } else {
-        const int hw = p.rope.gh * p.rope.gw;
-        const int f = i / hw;
-        const int rem = i - f * hw;
-        const int y = rem / p.rope.gw;
-        pos[0] = static_cast<int>((p.round + c) * p.rope.F + f);
-        pos[1] = y;
-        pos[2] = rem - y * p.rope.gw;
+    float gq[8], gk[8];
+    {
+        const float4 *gq4 = reinterpret_cast<const float4 *>(p.gamma_q + hh * D + part * 8);
+        const float4 *gk4 = reinterpret_cast<const float4 *>(p.gamma_k + hh * D + part * 8);
+        const float4 a = __ldg(gq4), b = __ldg(gq4 + 1), c = __ldg(gk4), d = __ldg(gk4 + 1);
+        gq[0] = a.x; gq[1] = a.y; gq[2] = a.z; gq[3] = a.w;
+        gq[4] = b.x; gq[5] = b.y; gq[6] = b.z; gq[7] = b.w;
+        gk[0] = c.x; gk[1] = c.y; gk[2] = c.z; gk[3] = c.w;
+        gk[4] = d.x; gk[5] = d.y; gk[6] = d.z; gk[7] = d.w;
     }
 
-    float xq[8], xk[8];
-    unpack8(uq, xq);
-    unpack8(uk, xk);
-    float ssq = 0.f, ssk = 0.f;
+    uint4 uq[kTokens], uk[kTokens], uv[kTokens];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        ssq = fmaf(xq[e], xq[e], ssq);
-        ssk = fmaf(xk[e], xk[e], ssk);
+    for (int tl = 0; tl < kTokens; ++tl) {
+        const long n = n0 + tl;
+        if (active && n < T) {
+            const long off = (n * p.H + h) * D + part * 8;
+            uq[tl] = __ldcs(reinterpret_cast<const uint4 *>(p.q + off));
+            uk[tl] = __ldcs(reinterpret_cast<const uint4 *>(p.k + off));
+            uv[tl] = __ldcs(reinterpret_cast<const uint4 *>(p.v + off));
+        } else {
+            uq[tl] = uk[tl] = uv[tl] = make_uint4(0u, 0u, 0u, 0u);
+        }
     }
+
 #pragma unroll
-    for (int o = TPR / 2; o > 0; o >>= 1) {
-        ssq += __shfl_xor_sync(mask, ssq, o);
-        ssk += __shfl_xor_sync(mask, ssk, o);
-    }
-    const float rq = rsqrtf(ssq * (1.0f / D) + p.eps);
-    const float rk = rsqrtf(ssk * (1.0f / D) + p.eps);
-
-    const float4 *gq4 = reinterpret_cast<const float4 *>(p.gamma_q + h * D + part * 8);
-    const float4 *gk4 = reinterpret_cast<const float4 *>(p.gamma_k + h * D + part * 8);
-    const float4 gq0 = __ldg(gq4), gq1 = __ldg(gq4 + 1);
-    const float4 gk0 = __ldg(gk4), gk1 = __ldg(gk4 + 1);
-    const float gq[8] = {gq0.x, gq0.y, gq0.z, gq0.w, gq1.x, gq1.y, gq1.z, gq1.w};
-    const float gk[8] = {gk0.x, gk0.y, gk0.z, gk0.w, gk1.x, gk1.y, gk1.z, gk1.w};
-
-    float yq[8], yk[8];
+    for (int tl = 0; tl < kTokens; ++tl) {
+        const long n = n0 + tl;
+        if (n >= T) break;                    // uniform across the block
+        float xq[8], xk[8];
+        unpack8(uq[tl], xq);
+        unpack8(uk[tl], xk);
+        float ssq = 0.f, ssk = 0.f;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const int pr = part * 4 + e;           // channel pair index
-        const int ax = s_axis[pr];
-        const int pv = ax == 0 ? pos[0] : (ax == 1 ? pos[1] : pos[2]);
-        const float ang = static_cast<float>(pv) * s_omega[pr];
-        float sn, cs;
-        sincosf(ang, &sn, &cs);
-        const float q0 = xq[2 * e] * rq * gq[2 * e], q1 = xq[2 * e + 1] * rq * gq[2 * e + 1];
-        const float k0 = xk[2 * e] * rk * gk[2 * e], k1 = xk[2 * e + 1] * rk * gk[2 * e + 1];
-        yq[2 * e] = q0 * cs - q1 * sn;
-        yq[2 * e + 1] = q0 * sn + q1 * cs;
-        yk[2 * e] = k0 * cs - k1 * sn;
-        yk[2 * e + 1] = k0 * sn + k1 * cs;
+        for (int e = 0; e < 8; ++e) {
+            ssq = fmaf(xq[e], xq[e], ssq);
+            ssk = fmaf(xk[e], xk[e], ssk);
+        }
+#pragma unroll
+        for (int o = TPR / 2; o > 0; o >>= 1) {
+            ssq += __shfl_xor_sync(0xFFFFFFFFu, ssq, o);
+            ssk += __shfl_xor_sync(0xFFFFFFFFu, ssk, o);
+        }
+        const float rq = rsqrtf(ssq * (1.0f / D) + p.eps);
+        const float rk = rsqrtf(ssk * (1.0f / D) + p.eps);
+        float yq[8], yk[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 cs = s_cs[tl][part * 4 + e];
+            const float q0 = xq[2 * e] * rq * gq[2 * e], q1 = xq[2 * e + 1] * rq * gq[2 * e + 1];
+            const float k0 = xk[2 * e] * rk * gk[2 * e], k1 = xk[2 * e + 1] * rk * gk[2 * e + 1];
+            yq[2 * e] = q0 * cs.x - q1 * cs.y;
+            yq[2 * e + 1] = q0 * cs.y + q1 * cs.x;
+            yk[2 * e] = k0 * cs.x - k1 * cs.y;
+            yk[2 * e + 1] = k0 * cs.y + k1 * cs.x;
+        }
+        if (active) {
+            const long off = (n * p.H + h) * D + part * 8;
+            const long coff = s_off[tl] + static_cast<long>(h) * D + part * 8;
+            *reinterpret_cast<uint4 *>(p.q_out + off) = pack8(yq);
+            *reinterpret_cast<uint4 *>(p.k_cache + coff) = pack8(yk);
+            *reinterpret_cast<uint4 *>(p.v_cache + coff) = uv[tl];
+        }
     }
-
-    const int slot = ring_slot(p.round + c, p.R);
-    const long coff = ((static_cast<long>(slot) * p.L + i) * p.H + h) * D + part * 8;
-    *reinterpret_cast<uint4 *>(p.q_out + off) = pack8(yq);
-    *reinterpret_cast<uint4 *>(p.k_cache + coff) = pack8(yk);
-    *reinterpret_cast<uint4 *>(p.v_cache + coff) = uv;
 }
 
 }  // namespace
 
-cudaError_t launch_append(const AppendParams &p, int D, cudaStream_t stream)
+cudaError_t launch_append(const AppendParams &p_in, int D, cudaStream_t stream)
 {
-    const long items = static_cast<long>(p.W) * p.L * p.H * (D / 8);
-    const int threads = 256;
-    const long blocks = (items + threads - 1) / threads;
-    if (blocks <= 0) return cudaSuccess;
+    AppendParams p = p_in;
+    const int tpr = D / 8;
+    const int groups = (p.H * tpr + kMaxThreads - 1) / kMaxThreads;
+    p.heads_per_block = (p.H + groups - 1) / groups;
+    const int threads = (p.heads_per_block * tpr + 31) / 32 * 32;
+    const long T = static_cast<long>(p.W) * p.L;
+    const long bx = (T + kTokens - 1) / kTokens;
+    const int by = (p.H + p.heads_per_block - 1) / p.heads_per_block;
+    if (bx <= 0) return cudaSuccess;
+    const dim3 grid(static_cast<unsigned>(bx), static_cast<unsigned>(by));
     if (D == 128)
-        qk_norm_rope_append_kernel<128><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(p);
+        qk_norm_rope_append_kernel<128><<<grid, threads, 0, stream>>>(p);
     else
-        qk_norm_rope_append_kernel<64><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(p);
+        qk_norm_rope_append_kernel<64><<<grid, threads, 0, stream>>>(p);
     return cudaGetLastError();
 }
 

@@ -8,24 +8,33 @@
 // masked tiles are never loaded, and the only element mask is "key row < L" in
 // the last 128-key tile of each chunk (TMA fills the rows past L with zeros).
 //
-// Work unit = (wave chunk c, head h, pair of 128-row query tiles).  One CTA per
-// SM walks units in longest-first order (cost (h_valid + c + 1) key chunks).
-// Warp roles (320 threads):
-//   warps 0-3  softmax for query tile 0 (TMEM lanes 0..127, one row per thread)
-//   warps 4-7  softmax for query tile 1
-//   warp  8    TMA producer: Q tiles, then K_j, V_j into a ring of smem stages
-//   warp  9    MMA issuer (one thread): S_x = Q_x K_j^T, O_x += P_x V_j
+// Work unit = (wave chunk c, head h, pair of 128-row query tiles).  Units are
+// numbered longest first (cost (h_valid + c + 1) key chunks); one CTA per SM
+// pops them from a global counter (greedy longest-processing-time order).
+// Warp roles (384 threads, three warpgroups):
+//   warps 0-3   softmax for query tile 0 (TMEM lanes 0..127, one row per thread)
+//   warps 4-7   softmax for query tile 1
+//   warp  8     scheduler + TMA producer: Q tiles, then K_j, V_j into a smem ring
+//   warp  9     MMA issuer (one thread): S_x = Q_x K_j^T, O_x += P_x V_j
+//   warps 10-11 idle (they only give their registers to the softmax warpgroups)
+// Registers: launched at 168 per thread; the control warpgroup drops to 88 and
+// the two softmax warpgroups rise to 208 (setmaxnreg), which is exactly the
+// launch pool.  The host refuses to launch if the compiled kernel does not use
+// 168 registers, so the increase can always be met.
 // TMEM (512 columns): S0 | S1 | O0 | O1.  Softmax overwrites the first half of
 // S_x with P_x (bf16 pairs) and the PV product reads P straight from TMEM.
 // The two query tiles ping-pong: while one warpgroup exponentiates, the tensor
 // core runs the other tile's PV and next QK^T.  Online softmax works in the
 // log2 domain and rescales O only when a row maximum grows by more than 2^8.
+// One score pair in four is exponentiated on the FMA pipe (Cody-Waite split and
+// a Remez polynomial, exp2_poly.h) to offload the MUFU unit.
 //
 // Every mbarrier wait is bounded (clock64 limit); on expiry the kernel records
 // kStatusTimeout in the plan's status word, all roles leave their loops, wait
 // for their own copies/MMAs in flight, and the CTA frees TMEM and returns.
 #include <cuda_bf16.h>
 
+#include "exp2_poly.h"
 #include "sm100.cuh"
 #include "wf_internal.h"
 
@@ -35,11 +44,16 @@ namespace {
 
 constexpr int BM = 128;              // query rows per tile
 constexpr int BN = 128;              // keys per tile
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
+constexpr uint32_t kRegsLaunch = 168, kRegsSoftmax = 208, kRegsControl = 88;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl == kThreads * kRegsLaunch,
+              "the register re-split must add up to the launch pool");
+constexpr int kSoftmaxWarpsArrive = 8;      // sched_empty: one arrival per softmax warp
+constexpr int kEmulatePeriod = 4;           // pair e uses the FMA-pipe exp2 when e % 4 == 3
 
 template <int D>
 struct Cfg {
@@ -50,7 +64,7 @@ struct Cfg {
     static constexpr uint32_t kQOff = 0;
     static constexpr uint32_t kKVOff = 2 * kTileBytes;
     static constexpr uint32_t kBarOff = kKVOff + kStages * kTileBytes;
-    static constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;
+    static constexpr uint32_t kSmemBytes = kBarOff + 512 + 1024;
     static constexpr uint32_t kS0 = 0, kS1 = 128, kO0 = 256, kO1 = 256 + D;
 };
 
@@ -58,13 +72,14 @@ struct Cfg {
 template <int S>
 struct Bars {
     static constexpr int q_full = 0, q_empty = 1, s_full = 2, p_ready = 4, o_final = 6,
-                         drain = 8, kv_full = 9, kv_empty = 9 + S, count = 9 + 2 * S;
+                         drain = 8, sched_full = 9, sched_empty = 11, kv_full = 13,
+                         kv_empty = 13 + S, count = 13 + 2 * S;
 };
 
 // Wait-site codes recorded in DeviceWords::timeout_where.
 enum : uint32_t {
     kWhereProducerQ = 1, kWhereProducerKV = 2, kWhereMmaQ = 3, kWhereMmaKV = 4,
-    kWhereMmaP = 5, kWhereSoftS = 6, kWhereSoftO = 7, kWhereDrain = 8,
+    kWhereMmaP = 5, kWhereSoftS = 6, kWhereSoftO = 7, kWhereDrain = 8, kWhereSched = 9,
 };
 
 struct Ctl {
@@ -96,6 +111,7 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ct
 
 struct Unit {
     int c, h, pair, n_kt;
+    bool has1;                                // query tile 1 holds rows of the chunk
 };
 
 __device__ __forceinline__ Unit decode_unit(const AttnParams &p, int u)
@@ -108,18 +124,24 @@ __device__ __forceinline__ Unit decode_unit(const AttnParams &p, int u)
     r.h = rem / p.n_qpairs;
     r.pair = rem - r.h * p.n_qpairs;
     r.n_kt = (p.h_valid + r.c + 1) * p.n_ktiles;
+    r.has1 = (2 * r.pair + 1) * BM < p.L;
     return r;
 }
 
+// The descriptors of one operand tile differ only in the start-address field
+// (low 14 bits), so they are built from a 32-bit low word and a constant high
+// word: fewer live 64-bit values in the MMA-issuing thread.
 template <int D>
 __device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t q_smem, uint32_t k_smem)
 {
     constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, false);
+    constexpr uint32_t hi = sw128_desc_hi(1024);
+    const uint32_t qlo = sw128_desc_lo(q_smem, 16), klo = sw128_desc_lo(k_smem, 16);
 #pragma unroll
     for (int s = 0; s < D / 16; ++s) {
-        const uint32_t off = (s >> 2) * Cfg<D>::kHalfBytes + (s & 3) * 32;
-        umma_ss(s_tmem, sw128_desc(q_smem + off, 16, 1024), sw128_desc(k_smem + off, 16, 1024),
-                idesc, s > 0 ? 1u : 0u);
+        const uint32_t off = ((s >> 2) * Cfg<D>::kHalfBytes + (s & 3) * 32) >> 4;
+        umma_ss(s_tmem, desc_join(qlo + off, hi), desc_join(klo + off, hi), idesc,
+                s > 0 ? 1u : 0u);
     }
 }
 
@@ -128,13 +150,39 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint3
                                          bool accumulate)
 {
     constexpr uint32_t idesc = idesc_bf16_f32(BM, D, true);
+    constexpr uint32_t hi = sw128_desc_hi(1024);
+    // V tile: 16 keys per step = 2 eight-row groups of 128 bytes; the two
+    // 64-channel halves of D sit kHalfBytes apart (leading byte offset).
+    const uint32_t vlo = sw128_desc_lo(v_smem, Cfg<D>::kHalfBytes);
 #pragma unroll
-    for (int s = 0; s < BN / 16; ++s) {
-        // V tile: 16 keys per step = 2 eight-row groups of 128 bytes; the two
-        // 64-channel halves of D sit kHalfBytes apart (leading byte offset).
-        umma_ts(o_tmem, p_tmem + s * 8, sw128_desc(v_smem + s * 2048, Cfg<D>::kHalfBytes, 1024),
-                idesc, (accumulate || s > 0) ? 1u : 0u);
-    }
+    for (int s = 0; s < BN / 16; ++s)
+        umma_ts(o_tmem, p_tmem + s * 8, desc_join(vlo + ((s * 2048) >> 4), hi), idesc,
+                (accumulate || s > 0) ? 1u : 0u);
+}
+
+// 2^x for a pair of scores on the FMA pipe: j = round(x) by the 1.5*2^23 shift,
+// f = x - j in [-1/2, 1/2], 2^f from the Remez polynomial, then j added to the
+// exponent field.  x is clamped at -126 so the exponent never wraps; inputs
+// below that (masked columns, deep underflow) give 2^-126 instead of 0, which
+// is below one fp32 ulp of the row sum (>= 1) and multiplies a zero V row.
+__device__ __forceinline__ void exp2_fma_pair(float x0, float x1, float &p0, float &p1)
+{
+    constexpr float kShift = 12582912.0f;   // 1.5 * 2^23
+    x0 = fmaxf(x0, -126.0f);
+    x1 = fmaxf(x1, -126.0f);
+    const uint64_t x = f2_pack(x0, x1);
+    const uint64_t t = f2_add(x, f2_pack(kShift, kShift));
+    const uint64_t jf = f2_add(t, f2_pack(-kShift, -kShift));
+    const uint64_t f = f2_fma(jf, f2_pack(-1.0f, -1.0f), x);
+    uint64_t q = f2_fma(f2_pack(kExp2C3, kExp2C3), f, f2_pack(kExp2C2, kExp2C2));
+    q = f2_fma(q, f, f2_pack(kExp2C1, kExp2C1));
+    q = f2_fma(q, f, f2_pack(kExp2C0, kExp2C0));
+    float q0, q1, t0, t1;
+    f2_unpack(q, q0, q1);
+    f2_unpack(t, t0, t1);
+    // the low bits of t hold j; (bits(t) << 23) == (j << 23) modulo 2^32
+    p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+    p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
 template <int D>
@@ -157,6 +205,7 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
     auto bar = [&](int i) -> uint32_t { return sbar + 8u * static_cast<uint32_t>(i); };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kBarOff + 8 * B::count);
     volatile uint32_t *abort_flag = tmem_slot + 1;
+    volatile int *sched_unit = reinterpret_cast<volatile int *>(tmem_slot + 2);   // [2]
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -168,6 +217,8 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
             mbar_init(bar(B::s_full + x), 1);
             mbar_init(bar(B::p_ready + x), 128);
             mbar_init(bar(B::o_final + x), 1);
+            mbar_init(bar(B::sched_full + x), 1);
+            mbar_init(bar(B::sched_empty + x), 1 + kSoftmaxWarpsArrive);
         }
         mbar_init(bar(B::drain), 1);
         for (int s = 0; s < S; ++s) {
@@ -187,21 +238,29 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
     const uint32_t tmem = *tmem_slot;
     const Ctl ctl{abort_flag, p.words, p.wait_limit};
 
-    if (warp == kProducerWarp) {
-        if (lane == 0) {
+    if (warp >= 8) {
+        regs_dec<kRegsControl>();
+        if (warp == kProducerWarp && lane == 0) {
+            // ---------------- scheduler + TMA producer ----------------
             tma_prefetch_desc(&tmap_q);
             tma_prefetch_desc(&tmap_k);
             tma_prefetch_desc(&tmap_v);
             uint32_t stage = 0, kv_phase = 0, q_phase = 0;
             uint32_t q_fills = 0, kv_fills = 0;   // copies issued so far
             bool ok = true;
-            for (int u = blockIdx.x; ok && u < p.n_units; u += gridDim.x) {
+            for (uint32_t it = 0; ok; ++it) {
+                const uint32_t sl = it & 1u, ph = (it >> 1) & 1u;
+                if (!(ok = wait_bar(bar(B::sched_empty + sl), ph ^ 1u, ctl, kWhereSched))) break;
+                const int u = static_cast<int>(atomicAdd(&p.words->sched_counter, 1u));
+                sched_unit[sl] = u;
+                mbar_arrive(bar(B::sched_full + sl));
+                if (u >= p.n_units) break;
                 const Unit un = decode_unit(p, u);
                 if (!(ok = wait_bar(bar(B::q_empty), q_phase ^ 1u, ctl, kWhereProducerQ))) break;
                 q_phase ^= 1u;
-                mbar_arrive_expect_tx(bar(B::q_full), 2 * C::kTileBytes);
+                mbar_arrive_expect_tx(bar(B::q_full), (un.has1 ? 2 : 1) * C::kTileBytes);
                 ++q_fills;
-                for (int x = 0; x < 2; ++x)
+                for (int x = 0; x < (un.has1 ? 2 : 1); ++x)
                     for (int hf = 0; hf < C::kHalves; ++hf)
                         tma_load_4d(sq + x * C::kTileBytes + hf * C::kHalfBytes, &tmap_q,
                                     bar(B::q_full), hf * 64, un.h, (2 * un.pair + x) * BM, un.c);
@@ -231,9 +290,8 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     if (f) wait_bar(bar(B::kv_full + s), (f - 1) & 1u, ctl, kWhereDrain, true);
                 }
             }
-        }
-    } else if (warp == kMmaWarp) {
-        if (lane == 0) {
+        } else if (warp == kMmaWarp && lane == 0) {
+            // ---------------- MMA issuer ----------------
             uint32_t stage = 0, kv_phase = 0, q_phase = 0;
             uint32_t p_phase[2] = {0u, 0u};
             const uint32_t tS[2] = {tmem + C::kS0, tmem + C::kS1};
@@ -245,7 +303,12 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
     ((st) = stage,                                                                     \
      ok = wait_bar(bar(B::kv_full + stage), kv_phase, ctl, kWhereMmaKV),               \
      (++stage == S ? (stage = 0, kv_phase ^= 1u) : 0u), tc_fence_after(), ok)
-            for (int u = blockIdx.x; ok && u < p.n_units; u += gridDim.x) {
+            for (uint32_t it = 0; ok; ++it) {
+                const uint32_t sl = it & 1u, ph = (it >> 1) & 1u;
+                if (!(ok = wait_bar(bar(B::sched_full + sl), ph, ctl, kWhereSched))) break;
+                const int u = sched_unit[sl];
+                mbar_arrive(bar(B::sched_empty + sl));
+                if (u >= p.n_units) break;
                 const Unit un = decode_unit(p, u);
                 if (!(ok = wait_bar(bar(B::q_full), q_phase, ctl, kWhereMmaQ))) break;
                 q_phase ^= 1u;
@@ -253,8 +316,10 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 if (!WF_NEXT_STAGE(kst)) break;
                 issue_qk<D>(tS[0], sQ[0], skv + kst * C::kTileBytes);
                 umma_commit(bar(B::s_full + 0));
-                issue_qk<D>(tS[1], sQ[1], skv + kst * C::kTileBytes);
-                umma_commit(bar(B::s_full + 1));
+                if (un.has1) {
+                    issue_qk<D>(tS[1], sQ[1], skv + kst * C::kTileBytes);
+                    umma_commit(bar(B::s_full + 1));
+                }
                 umma_commit(bar(B::kv_empty + kst));
                 if (un.n_kt == 1) umma_commit(bar(B::q_empty));
                 for (int j = 0; ok && j < un.n_kt; ++j) {
@@ -274,17 +339,22 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                         umma_commit(bar(B::o_final + 0));
                     }
                     // query tile 1
-                    if (!(ok = wait_bar(bar(B::p_ready + 1), p_phase[1], ctl, kWhereMmaP))) break;
-                    p_phase[1] ^= 1u;
-                    tc_fence_after();
-                    issue_pv<D>(tO[1], tS[1], skv + vst * C::kTileBytes, j > 0);
+                    if (un.has1) {
+                        if (!(ok = wait_bar(bar(B::p_ready + 1), p_phase[1], ctl, kWhereMmaP)))
+                            break;
+                        p_phase[1] ^= 1u;
+                        tc_fence_after();
+                        issue_pv<D>(tO[1], tS[1], skv + vst * C::kTileBytes, j > 0);
+                    }
                     umma_commit(bar(B::kv_empty + vst));
                     if (more) {
-                        issue_qk<D>(tS[1], sQ[1], skv + kst2 * C::kTileBytes);
-                        umma_commit(bar(B::s_full + 1));
+                        if (un.has1) {
+                            issue_qk<D>(tS[1], sQ[1], skv + kst2 * C::kTileBytes);
+                            umma_commit(bar(B::s_full + 1));
+                        }
                         umma_commit(bar(B::kv_empty + kst2));
                         if (j + 2 == un.n_kt) umma_commit(bar(B::q_empty));
-                    } else {
+                    } else if (un.has1) {
                         umma_commit(bar(B::o_final + 1));
                     }
                 }
@@ -295,6 +365,7 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
             wait_bar(bar(B::drain), 0u, ctl, kWhereDrain, true);
         }
     } else {
+        regs_inc<kRegsSoftmax>();
         // ---------------- softmax warpgroups ----------------
         const int x = warp >> 2;                    // query tile of this warpgroup
         const int row = threadIdx.x & 127;          // TMEM lane = row of the tile
@@ -302,10 +373,20 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
         const uint32_t tS = tmem + lane_sel + (x ? C::kS1 : C::kS0);
         const uint32_t tO = tmem + lane_sel + (x ? C::kO1 : C::kO0);
         const float scale = p.scale_log2;
+        const uint64_t sc2 = f2_pack(scale, scale);
         uint32_t s_phase = 0, o_phase = 0;
         bool ok = true;
-        for (int u = blockIdx.x; ok && u < p.n_units; u += gridDim.x) {
+        for (uint32_t it = 0; ok; ++it) {
+            const uint32_t sl = it & 1u, ph = (it >> 1) & 1u;
+            ok = wait_bar(bar(B::sched_full + sl), ph, ctl, kWhereSched);
+            ok = __all_sync(0xFFFFFFFFu, ok);
+            if (!ok) break;
+            const int u = sched_unit[sl];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B::sched_empty + sl));
+            if (u >= p.n_units) break;
             const Unit un = decode_unit(p, u);
+            if (x == 1 && !un.has1) continue;       // the tile lies past the chunk's end
             const int q_row = (2 * un.pair + x) * BM + row;     // row inside chunk c
             float m_run = -INFINITY, l_run = 0.f;
             for (int j = 0; j < un.n_kt; ++j) {
@@ -320,16 +401,19 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 tmem_wait_ld();
                 const int t = j % p.n_ktiles;
                 const int valid = t == p.n_ktiles - 1 ? p.L - t * BN : BN;
-                float mx = -INFINITY;
+                if (valid < BN) {                   // last tile of a chunk: rows >= L
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
+                    for (int q4 = 0; q4 < 4; ++q4)
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        float s = __uint_as_float(r[q4][e]);
-                        if (q4 * 32 + e >= valid) s = -INFINITY;
-                        r[q4][e] = __float_as_uint(s);
-                        mx = fmaxf(mx, s);
-                    }
+                        for (int e = 0; e < 32; ++e)
+                            if (q4 * 32 + e >= valid) r[q4][e] = __float_as_uint(-INFINITY);
+                }
+                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                for (int k = 0; k < 64; ++k)
+                    mx4[k & 3] = fmax3(mx4[k & 3], __uint_as_float(r[k >> 4][(2 * k) & 31]),
+                                       __uint_as_float(r[k >> 4][(2 * k + 1) & 31]));
+                const float mx = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
                 // The row maximum only moves forward when it grew by more than
                 // 2^8: otherwise exponents stay <= 2^8 against the stale maximum
                 // and O keeps its scale.  (At j = 0 PV overwrites O.)
@@ -340,8 +424,8 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     l_run *= alpha;
                     m_run = m_new;
                 }
-                const float neg_m = -m_run;
-                float sum = 0.f;
+                const uint64_t nm2 = f2_pack(-m_run, -m_run);
+                uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     // P columns [64*hf, 64*hf + 64) -> packed bf16 TMEM columns [32*hf, 32*hf + 32)
@@ -349,14 +433,25 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const int col = 64 * hf + 2 * e;
-                        const float p0 = ex2_approx(fmaf(__uint_as_float(r[col >> 5][col & 31]), scale, neg_m));
-                        const float p1 = ex2_approx(fmaf(__uint_as_float(r[col >> 5][(col + 1) & 31]), scale, neg_m));
-                        sum += p0 + p1;
+                        const uint64_t s2 = f2_pack(__uint_as_float(r[col >> 5][col & 31]),
+                                                    __uint_as_float(r[col >> 5][(col + 1) & 31]));
+                        float x0, x1, p0, p1;
+                        f2_unpack(f2_fma(s2, sc2, nm2), x0, x1);
+                        if ((e % kEmulatePeriod) == kEmulatePeriod - 1) {
+                            exp2_fma_pair(x0, x1, p0, p1);
+                        } else {
+                            p0 = ex2_approx(x0);
+                            p1 = ex2_approx(x1);
+                        }
+                        acc[e & 3] = f2_add(acc[e & 3], f2_pack(p0, p1));
                         pk[e] = pack_bf16x2(p0, p1);
                     }
                     tmem_st32(tS + 32 * hf, pk);
                 }
-                l_run += sum;
+                float a0, a1, b0, b1;
+                f2_unpack(f2_add(acc[0], acc[1]), a0, a1);
+                f2_unpack(f2_add(acc[2], acc[3]), b0, b1);
+                l_run += (a0 + a1) + (b0 + b1);
                 if (j > 0 && __any_sync(0xFFFFFFFFu, need)) {
                     // O is quiescent here: the MMA that filled S_x(j) was issued
                     // after PV_x(j-1), and PV_x(j) waits for this warpgroup.
@@ -411,7 +506,10 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+    if (warp == kMmaWarp) {
+        __syncwarp();
+        tmem_dealloc(tmem, kTmemCols);
+    }
 }
 
 }  // namespace
@@ -421,8 +519,16 @@ static cudaError_t launch_attn_d(const CUtensorMap &mq, const CUtensorMap &mk, c
                                  const AttnParams &p, int grid, cudaStream_t stream)
 {
     const uint32_t smem = Cfg<D>::kSmemBytes;
-    cudaError_t e = cudaFuncSetAttribute(chunk_causal_attn_kernel<D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    // The setmaxnreg split assumes the kernel was compiled to exactly the
+    // launch budget; any other count could leave the increase waiting.
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, chunk_causal_attn_kernel<D>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != static_cast<int>(kRegsLaunch)) return cudaErrorInvalidKernelImage;
+    e = cudaFuncSetAttribute(chunk_causal_attn_kernel<D>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    e = cudaMemsetAsync(&p.words->sched_counter, 0, sizeof(uint32_t), stream);
     if (e != cudaSuccess) return e;
     chunk_causal_attn_kernel<D><<<grid, kThreads, smem, stream>>>(mq, mk, mv, p);
     return cudaGetLastError();

@@ -29,7 +29,7 @@ void fill_rope_table(wf::RopeParams &r, double theta)
     int pair = 0;
     for (int a = 0; a < 3; ++a)
         for (int i = 0; i < width[a] / 2; ++i, ++pair) {
-            r.omega[pair] = static_cast<float>(std::pow(theta, -2.0 * i / width[a]));
+            r.omega[pair] = std::pow(theta, -2.0 * i / width[a]);
             r.axis[pair] = static_cast<int8_t>(a);
         }
 }

@@ -52,7 +52,7 @@ struct DeviceWords {
 struct RopeParams {
     int dt, dh, dw;           // channel widths of the t / h / w blocks
     int F, gh, gw;            // chunk geometry for derived positions (F = 0: unset)
-    float omega[kMaxHeadDim / 2];   // per channel pair: theta^(-2i/d_axis)
+    double omega[kMaxHeadDim / 2];  // per channel pair: theta^(-2i/d_axis)
     int8_t axis[kMaxHeadDim / 2];   // per channel pair: 0 = t, 1 = h, 2 = w
 };
 
@@ -63,6 +63,7 @@ struct AppendParams {
     uint16_t *q_out, *k_cache, *v_cache;
     long round;
     int L, W, R, H;
+    int heads_per_block;      // heads covered by one block (blockIdx.y picks the group)
     float eps;
     RopeParams rope;
 };
