@@ -17,17 +17,20 @@
 //   warp  8     scheduler + TMA producer: Q tiles, then K_j, V_j into a smem ring
 //   warp  9     MMA issuer (one thread): S_x = Q_x K_j^T, O_x += P_x V_j
 //   warps 10-11 idle (they only give their registers to the softmax warpgroups)
-// Registers: launched at 168 per thread; the control warpgroup drops to 88 and
-// the two softmax warpgroups rise to 208 (setmaxnreg), which is exactly the
-// launch pool.  The host refuses to launch if the compiled kernel does not use
+// Registers: launched at 168 per thread; the control warpgroup drops to 104 and
+// the two softmax warpgroups rise to 200 (setmaxnreg), which is exactly the
+// launch pool and leaves both paths spill-free.  The host refuses to launch if the compiled kernel does not use
 // 168 registers, so the increase can always be met.
 // TMEM (512 columns): S0 | S1 | O0 | O1.  Softmax overwrites the first half of
 // S_x with P_x (bf16 pairs) and the PV product reads P straight from TMEM.
+// P is published in two halves of 64 keys: PV on the first half starts while
+// the softmax still exponentiates the second.
 // The two query tiles ping-pong: while one warpgroup exponentiates, the tensor
 // core runs the other tile's PV and next QK^T.  Online softmax works in the
 // log2 domain and rescales O only when a row maximum grows by more than 2^8.
-// One score pair in four is exponentiated on the FMA pipe (Cody-Waite split and
-// a Remez polynomial, exp2_poly.h) to offload the MUFU unit.
+// A fraction of the score pairs can be exponentiated on the FMA pipe
+// (Cody-Waite split and a Remez polynomial, exp2_poly.h) to offload MUFU; see
+// kEmulatePeriod.
 //
 // Every mbarrier wait is bounded (clock64 limit); on expiry the kernel records
 // kStatusTimeout in the plan's status word, all roles leave their loops, wait
@@ -49,11 +52,15 @@ constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
-constexpr uint32_t kRegsLaunch = 168, kRegsSoftmax = 208, kRegsControl = 88;
+constexpr uint32_t kRegsLaunch = 168, kRegsSoftmax = 200, kRegsControl = 104;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl == kThreads * kRegsLaunch,
               "the register re-split must add up to the launch pool");
 constexpr int kSoftmaxWarpsArrive = 8;      // sched_empty: one arrival per softmax warp
-constexpr int kEmulatePeriod = 4;           // pair e uses the FMA-pipe exp2 when e % 4 == 3
+// Pair e of a 32-pair block takes the FMA-pipe exp2 when e % kEmulatePeriod ==
+// kEmulatePeriod - 1; 0 keeps every exponential on MUFU.  Measured on B200 at
+// this design point the softmax is bound by issue and latency rather than by
+// MUFU throughput, so the default is 0 (all MUFU); 4 and 8 are tested too.
+constexpr int kEmulatePeriod = 0;
 
 template <int D>
 struct Cfg {
@@ -72,8 +79,8 @@ struct Cfg {
 template <int S>
 struct Bars {
     static constexpr int q_full = 0, q_empty = 1, s_full = 2, p_ready = 4, o_final = 6,
-                         drain = 8, sched_full = 9, sched_empty = 11, kv_full = 13,
-                         kv_empty = 13 + S, count = 13 + 2 * S;
+                         drain = 8, sched_full = 9, sched_empty = 11, p_half = 13, kv_full = 15,
+                         kv_empty = 15 + S, count = 15 + 2 * S;
 };
 
 // Wait-site codes recorded in DeviceWords::timeout_where.
@@ -145,9 +152,10 @@ __device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t q_smem, uint3
     }
 }
 
+// O += P V over keys [64*half, 64*half + 64) of the tile (4 steps of 16 keys).
 template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem,
-                                         bool accumulate)
+__device__ __forceinline__ void issue_pv_half(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem,
+                                              int half, bool accumulate)
 {
     constexpr uint32_t idesc = idesc_bf16_f32(BM, D, true);
     constexpr uint32_t hi = sw128_desc_hi(1024);
@@ -155,9 +163,11 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint3
     // 64-channel halves of D sit kHalfBytes apart (leading byte offset).
     const uint32_t vlo = sw128_desc_lo(v_smem, Cfg<D>::kHalfBytes);
 #pragma unroll
-    for (int s = 0; s < BN / 16; ++s)
+    for (int i = 0; i < BN / 32; ++i) {
+        const int s = half * (BN / 32) + i;
         umma_ts(o_tmem, p_tmem + s * 8, desc_join(vlo + ((s * 2048) >> 4), hi), idesc,
                 (accumulate || s > 0) ? 1u : 0u);
+    }
 }
 
 // 2^x for a pair of scores on the FMA pipe: j = round(x) by the 1.5*2^23 shift,
@@ -216,6 +226,7 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
         for (int x = 0; x < 2; ++x) {
             mbar_init(bar(B::s_full + x), 1);
             mbar_init(bar(B::p_ready + x), 128);
+            mbar_init(bar(B::p_half + x), 128);
             mbar_init(bar(B::o_final + x), 1);
             mbar_init(bar(B::sched_full + x), 1);
             mbar_init(bar(B::sched_empty + x), 1 + kSoftmaxWarpsArrive);
@@ -293,7 +304,7 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
         } else if (warp == kMmaWarp && lane == 0) {
             // ---------------- MMA issuer ----------------
             uint32_t stage = 0, kv_phase = 0, q_phase = 0;
-            uint32_t p_phase[2] = {0u, 0u};
+            uint32_t p_phase[2] = {0u, 0u};   // shared by p_half and p_ready (same cadence)
             const uint32_t tS[2] = {tmem + C::kS0, tmem + C::kS1};
             const uint32_t tO[2] = {tmem + C::kO0, tmem + C::kO1};
             const uint32_t sQ[2] = {sq, sq + C::kTileBytes};
@@ -326,11 +337,14 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     const bool more = j + 1 < un.n_kt;
                     uint32_t vst, kst2 = 0;
                     if (!WF_NEXT_STAGE(vst)) break;
-                    // query tile 0
+                    // query tile 0: PV over the first 64 keys as soon as that half of P landed
+                    if (!(ok = wait_bar(bar(B::p_half + 0), p_phase[0], ctl, kWhereMmaP))) break;
+                    tc_fence_after();
+                    issue_pv_half<D>(tO[0], tS[0], skv + vst * C::kTileBytes, 0, j > 0);
                     if (!(ok = wait_bar(bar(B::p_ready + 0), p_phase[0], ctl, kWhereMmaP))) break;
                     p_phase[0] ^= 1u;
                     tc_fence_after();
-                    issue_pv<D>(tO[0], tS[0], skv + vst * C::kTileBytes, j > 0);
+                    issue_pv_half<D>(tO[0], tS[0], skv + vst * C::kTileBytes, 1, true);
                     if (more) {
                         if (!WF_NEXT_STAGE(kst2)) break;
                         issue_qk<D>(tS[0], sQ[0], skv + kst2 * C::kTileBytes);
@@ -340,11 +354,15 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     }
                     // query tile 1
                     if (un.has1) {
+                        if (!(ok = wait_bar(bar(B::p_half + 1), p_phase[1], ctl, kWhereMmaP)))
+                            break;
+                        tc_fence_after();
+                        issue_pv_half<D>(tO[1], tS[1], skv + vst * C::kTileBytes, 0, j > 0);
                         if (!(ok = wait_bar(bar(B::p_ready + 1), p_phase[1], ctl, kWhereMmaP)))
                             break;
                         p_phase[1] ^= 1u;
                         tc_fence_after();
-                        issue_pv<D>(tO[1], tS[1], skv + vst * C::kTileBytes, j > 0);
+                        issue_pv_half<D>(tO[1], tS[1], skv + vst * C::kTileBytes, 1, true);
                     }
                     umma_commit(bar(B::kv_empty + vst));
                     if (more) {
@@ -424,34 +442,6 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     l_run *= alpha;
                     m_run = m_new;
                 }
-                const uint64_t nm2 = f2_pack(-m_run, -m_run);
-                uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    // P columns [64*hf, 64*hf + 64) -> packed bf16 TMEM columns [32*hf, 32*hf + 32)
-                    uint32_t pk[32];
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int col = 64 * hf + 2 * e;
-                        const uint64_t s2 = f2_pack(__uint_as_float(r[col >> 5][col & 31]),
-                                                    __uint_as_float(r[col >> 5][(col + 1) & 31]));
-                        float x0, x1, p0, p1;
-                        f2_unpack(f2_fma(s2, sc2, nm2), x0, x1);
-                        if ((e % kEmulatePeriod) == kEmulatePeriod - 1) {
-                            exp2_fma_pair(x0, x1, p0, p1);
-                        } else {
-                            p0 = ex2_approx(x0);
-                            p1 = ex2_approx(x1);
-                        }
-                        acc[e & 3] = f2_add(acc[e & 3], f2_pack(p0, p1));
-                        pk[e] = pack_bf16x2(p0, p1);
-                    }
-                    tmem_st32(tS + 32 * hf, pk);
-                }
-                float a0, a1, b0, b1;
-                f2_unpack(f2_add(acc[0], acc[1]), a0, a1);
-                f2_unpack(f2_add(acc[2], acc[3]), b0, b1);
-                l_run += (a0 + a1) + (b0 + b1);
                 if (j > 0 && __any_sync(0xFFFFFFFFu, need)) {
                     // O is quiescent here: the MMA that filled S_x(j) was issued
                     // after PV_x(j-1), and PV_x(j) waits for this warpgroup.
@@ -466,9 +456,39 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                         tmem_st32(tO + cc * 32, o);
                     }
                 }
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(bar(B::p_ready + x));
+                const uint64_t nm2 = f2_pack(-m_run, -m_run);
+                uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    // P columns [64*hf, 64*hf + 64) -> packed bf16 TMEM columns [32*hf, 32*hf + 32)
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int col = 64 * hf + 2 * e;
+                        const uint64_t s2 = f2_pack(__uint_as_float(r[col >> 5][col & 31]),
+                                                    __uint_as_float(r[col >> 5][(col + 1) & 31]));
+                        float x0, x1, p0, p1;
+                        f2_unpack(f2_fma(s2, sc2, nm2), x0, x1);
+                        if (kEmulatePeriod > 0 && (e % (kEmulatePeriod > 0 ? kEmulatePeriod : 1)) ==
+                                                      kEmulatePeriod - 1) {
+                            exp2_fma_pair(x0, x1, p0, p1);
+                        } else {
+                            p0 = ex2_approx(x0);
+                            p1 = ex2_approx(x1);
+                        }
+                        acc[e & 3] = f2_add(acc[e & 3], f2_pack(p0, p1));
+                        pk[e] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st32(tS + 32 * hf, pk);
+                    // publish this half of P (and any rescale of O before it)
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(bar(hf == 0 ? B::p_half + x : B::p_ready + x));
+                }
+                float a0, a1, b0, b1;
+                f2_unpack(f2_add(acc[0], acc[1]), a0, a1);
+                f2_unpack(f2_add(acc[2], acc[3]), b0, b1);
+                l_run += (a0 + a1) + (b0 + b1);
             }
             if (!ok) break;
             ok = wait_bar(bar(B::o_final + x), o_phase, ctl, kWhereSoftO);
