@@ -39,6 +39,7 @@ SIGNATURES = {
     "wf_sync_status": (_I, [_P, _P]),
     "wf_plan_debug_ranges": (_I, [_P, _L, _P, _I]),
     "wf_status_string": (ctypes.c_char_p, [_I]),
+    "wf_chunk_causal_attn_noalloc": (_I, [_I, _I, _I, _I, _I, _L, _P, _P, _P, _P, _P, _P]),
 }
 
 _lib = None
@@ -188,3 +189,15 @@ def wf_plan_debug_ranges(plan: Plan, round_: int):
     buf = (ctypes.c_int32 * (4 * max(n, 1)))()
     lib.wf_plan_debug_ranges(plan.handle, round_, buf, n)
     return [tuple(buf[4 * i:4 * i + 4]) for i in range(n)]
+
+
+def wf_chunk_causal_attn_noalloc(chunk_tokens, n_wave_chunks, n_hist_chunks, heads, head_dim,
+                                 round_, q_out, k_cache, v_cache, o, lse=None,
+                                 stream=None) -> None:
+    """Attention without a plan, for callers that must not allocate device memory
+    (see include/wf.h): the kernel's scratch lives in a block compiled into the
+    library, shared by every call on the device."""
+    _check(load().wf_chunk_causal_attn_noalloc(chunk_tokens, n_wave_chunks, n_hist_chunks,
+                                               heads, head_dim, round_, _ptr(q_out),
+                                               _ptr(k_cache), _ptr(v_cache), _ptr(o), _ptr(lse),
+                                               _stream(stream)), "wf_chunk_causal_attn_noalloc")

@@ -143,6 +143,29 @@ WF_API int wf_plan_debug_ranges(wf_plan_t plan, long round, int32_t *out, int ca
 
 WF_API const char *wf_status_string(int status);
 
+/* Chunk-causal attention of round r without a plan, for callers that must not
+ * allocate device memory (for example a serving loop whose device memory is
+ * owned by a framework's caching allocator or reserved up front, where a
+ * direct cudaMalloc would break that accounting or stall the device).  The
+ * paper has no counterpart: this is an interface choice of this library.
+ * Same computation, layouts, alignment rules and shape limits as wf_plan +
+ * wf_chunk_causal_attn; the shape is passed directly.  Instead of the plan's
+ * device block the kernel's scratch (status word, timeout site, work counter)
+ * lives in a 256-byte block compiled into the library, present on every GPU
+ * that loads it until the process exits; no cudaMalloc, cudaFree or
+ * allocating library call is made.  The first call on a device looks up that
+ * block's device address (cudaGetSymbolAddress); make that first call before
+ * any stream capture.  All calls on a device share the block: each clears what
+ * must start at zero on its own stream, and calls that overlap on the GPU race
+ * on it.  A device-side timeout is recorded in the block but not reported
+ * here.  Returns WF_OK, WF_ERR_INVALID_ARG / WF_ERR_UNSUPPORTED for shapes or
+ * pointers the plan API would reject, WF_ERR_NO_DEVICE, WF_ERR_DEVICE or
+ * WF_ERR_CUDA. */
+WF_API int wf_chunk_causal_attn_noalloc(int chunk_tokens, int n_wave_chunks, int n_hist_chunks,
+                                        int heads, int head_dim, long round,
+                                        const void *q_out, const void *k_cache,
+                                        const void *v_cache, void *o, float *lse, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
