@@ -52,6 +52,10 @@ constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
+// Waits for this CTA's own copies and MMAs in flight before it releases smem
+// and TMEM use this fixed limit, not the plan's (which tests may set tiny):
+// those operations always complete, so the drain only has to outlast them.
+constexpr unsigned long long kDrainLimit = 1ull << 32;
 constexpr uint32_t kRegsLaunch = 168, kRegsSoftmax = 200, kRegsControl = 104;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl == kThreads * kRegsLaunch,
               "the register re-split must add up to the launch pool");
@@ -96,18 +100,20 @@ struct Ctl {
 };
 
 // Bounded wait on one mbarrier phase.  Returns false on timeout or when another
-// role already aborted (unless `drain`, which ignores the abort flag).
+// role already aborted (unless `drain`, which ignores the abort flag and waits
+// up to kDrainLimit).
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ctl &ctl,
                                          uint32_t where, bool drain = false)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
+    const unsigned long long limit = drain ? kDrainLimit : ctl.limit;
     while (true) {
 #pragma unroll 1
         for (int k = 0; k < 32; ++k)
             if (mbar_try_wait(bar, parity)) return true;
         if (!drain && *ctl.abort) return false;
-        if (static_cast<unsigned long long>(clock64() - t0) > ctl.limit) {
+        if (static_cast<unsigned long long>(clock64() - t0) > limit) {
             *ctl.abort = 1u;
             atomicOr(&ctl.words->status, kStatusTimeout);
             atomicCAS(&ctl.words->timeout_where, 0u, where);
@@ -258,6 +264,7 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
             tma_prefetch_desc(&tmap_v);
             uint32_t stage = 0, kv_phase = 0, q_phase = 0;
             uint32_t q_fills = 0, kv_fills = 0;   // copies issued so far
+            bool withhold = p.withhold_q != 0;    // test hook: first Q copy never issued
             bool ok = true;
             for (uint32_t it = 0; ok; ++it) {
                 const uint32_t sl = it & 1u, ph = (it >> 1) & 1u;
@@ -269,12 +276,19 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 const Unit un = decode_unit(p, u);
                 if (!(ok = wait_bar(bar(B::q_empty), q_phase ^ 1u, ctl, kWhereProducerQ))) break;
                 q_phase ^= 1u;
-                mbar_arrive_expect_tx(bar(B::q_full), (un.has1 ? 2 : 1) * C::kTileBytes);
-                ++q_fills;
-                for (int x = 0; x < (un.has1 ? 2 : 1); ++x)
-                    for (int hf = 0; hf < C::kHalves; ++hf)
-                        tma_load_4d(sq + x * C::kTileBytes + hf * C::kHalfBytes, &tmap_q,
-                                    bar(B::q_full), hf * 64, un.h, (2 * un.pair + x) * BM, un.c);
+                if (withhold) {
+                    // nothing will ever complete this q_full phase: the MMA
+                    // thread's bounded wait must expire (tests only)
+                    withhold = false;
+                } else {
+                    mbar_arrive_expect_tx(bar(B::q_full), (un.has1 ? 2 : 1) * C::kTileBytes);
+                    ++q_fills;
+                    for (int x = 0; x < (un.has1 ? 2 : 1); ++x)
+                        for (int hf = 0; hf < C::kHalves; ++hf)
+                            tma_load_4d(sq + x * C::kTileBytes + hf * C::kHalfBytes, &tmap_q,
+                                        bar(B::q_full), hf * 64, un.h, (2 * un.pair + x) * BM,
+                                        un.c);
+                }
                 for (int j = 0; ok && j < un.n_kt; ++j) {
                     const int b = j / p.n_ktiles;
                     const int t = j - b * p.n_ktiles;

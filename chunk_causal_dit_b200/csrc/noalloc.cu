@@ -160,6 +160,7 @@ extern "C" int wf_chunk_causal_attn_noalloc(int chunk_tokens, int n_wave_chunks,
     a.n_units = heads * n_wave_chunks * n_qpairs;
     a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(head_dim)));
     a.wait_limit = 1ull << 32;
+    a.withhold_q = 0;
     a.o = static_cast<uint16_t *>(o);
     a.lse = lse;
     a.words = static_cast<wf::DeviceWords *>(scratch);

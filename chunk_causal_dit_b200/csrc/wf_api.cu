@@ -118,6 +118,7 @@ int wf_plan(int chunk_tokens, int n_wave_chunks, int n_hist_chunks, int heads, i
     p->rope.F = p->rope.gh = p->rope.gw = 0;
     fill_rope_table(p->rope, p->theta);
     p->wait_limit = kDefaultWaitLimit;
+    p->withhold_q = 0;
     p->device = -1;
     p->num_sms = 0;
     p->cc_major = p->cc_minor = 0;
@@ -183,6 +184,13 @@ int wf_plan_set_wait_limit(wf_plan_t p, unsigned long long cycles)
 {
     if (p == nullptr) return WF_ERR_INVALID_ARG;
     p->wait_limit = cycles == 0 ? kDefaultWaitLimit : cycles;
+    return WF_OK;
+}
+
+int wf_plan_set_withhold_q(wf_plan_t p, int on)
+{
+    if (p == nullptr) return WF_ERR_INVALID_ARG;
+    p->withhold_q = on ? 1 : 0;
     return WF_OK;
 }
 
@@ -281,6 +289,7 @@ int wf_chunk_causal_attn(wf_plan_t p, long round, const void *q_out, const void 
     a.n_units = p->H * p->W * a.n_qpairs;
     a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(p->D)));
     a.wait_limit = p->wait_limit;
+    a.withhold_q = p->withhold_q;
     a.o = static_cast<uint16_t *>(o);
     a.lse = lse;
     a.words = p->words;

@@ -77,6 +77,7 @@ struct AttnParams {
     int n_units;              // H * W * n_qpairs
     float scale_log2;         // log2(e) / sqrt(D)
     unsigned long long wait_limit;  // SM clock cycles
+    int withhold_q;           // test hook: withhold each CTA's first Q-tile copy
     uint16_t *o;
     float *lse;
     DeviceWords *words;
@@ -90,6 +91,7 @@ struct wf_plan_s {
     double eps;
     wf::RopeParams rope;
     unsigned long long wait_limit;
+    int withhold_q;           // test hook, see wf_plan_set_withhold_q
     int device;               // -1: no device state
     int num_sms;
     int cc_major, cc_minor;   // compute capability of `device`

@@ -31,6 +31,7 @@ SIGNATURES = {
     "wf_plan_set_rope_split": (_I, [_P, _I, _I, _I]),
     "wf_plan_set_norm_eps": (_I, [_P, ctypes.c_double]),
     "wf_plan_set_wait_limit": (_I, [_P, ctypes.c_ulonglong]),
+    "wf_plan_set_withhold_q": (_I, [_P, _I]),
     "wf_plan_destroy": (None, [_P]),
     "wf_cache_bytes": (ctypes.c_size_t, [_P]),
     "wf_useful_flops": (ctypes.c_double, [_P, _L]),
@@ -128,6 +129,11 @@ class Plan:
 
     def set_wait_limit(self, cycles: int):
         _check(load().wf_plan_set_wait_limit(self.handle, cycles), "wf_plan_set_wait_limit")
+        return self
+
+    def set_withhold_q(self, on: bool):
+        """Test hook: make the attention kernel's first Q wait expire (see wf.h)."""
+        _check(load().wf_plan_set_withhold_q(self.handle, int(bool(on))), "wf_plan_set_withhold_q")
         return self
 
     def destroy(self):

@@ -92,6 +92,14 @@ WF_API int wf_plan_set_norm_eps(wf_plan_t plan, double eps);
  * about two seconds).  Exposed so that tests can make a wait expire quickly. */
 WF_API int wf_plan_set_wait_limit(wf_plan_t plan, unsigned long long cycles);
 
+/* Test hook for failure detection, off by default.  With on != 0 the attention
+ * kernel's producer withholds the first Q-tile copy of every CTA, so the MMA
+ * warp's wait for it cannot complete: the bounded wait expires, the kernel
+ * stops cleanly (copies and MMAs in flight drained, TMEM freed) and
+ * wf_sync_status returns WF_ERR_TIMEOUT.  Nothing faults or traps; the
+ * context stays usable.  Pair it with a short wf_plan_set_wait_limit. */
+WF_API int wf_plan_set_withhold_q(wf_plan_t plan, int on);
+
 WF_API void wf_plan_destroy(wf_plan_t plan);
 
 /* Bytes of ONE ring (K or V): R * L * H * D * 2.  0 for a NULL plan. */
