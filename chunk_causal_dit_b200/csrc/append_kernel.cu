@@ -8,10 +8,11 @@
 // Memory-bound: 12*T*H*D bytes per call (read q, k, v; write q', K', V).
 // A block covers kTokens consecutive tokens for a group of heads.  Thread
 // (h, part) owns channels [8*part, 8*part + 8) of head h -- one 16-byte vector
-// per tensor -- and issues the loads of all kTokens tokens before computing.
+// per tensor -- and issues the loads of all kTokens tokens first.
 // The D/8 threads of a row reduce the sum of squares with shuffles; RoPE pairs
 // (2i, 2i+1) never straddle threads.  The rotation angles depend on the token
-// only, so each block computes them once per token in a prologue: the angle
+// only, so each block computes them once per token, while its loads are in
+// flight: the angle
 // pos * omega in fp64, reduced to [-pi, pi] in fp64, then fp32 sincos -- so the
 // fp32 error of the rotation stays a few ulps of the pair's length at any
 // position.
@@ -24,7 +25,7 @@ namespace wf {
 
 namespace {
 
-constexpr int kTokens = 4;         // tokens per block
+constexpr int kTokens = 2;         // tokens per block (measured best on B200: 2 > 3 > 1 > 4 > 8)
 constexpr int kMaxThreads = 512;   // threads per block (head groups split larger H)
 
 __device__ __forceinline__ void unpack8(const uint4 &u, float (&x)[8])
@@ -58,37 +59,7 @@ __global__ void __launch_bounds__(kMaxThreads) qk_norm_rope_append_kernel(const 
     const long T = static_cast<long>(p.W) * p.L;
     const long n0 = static_cast<long>(blockIdx.x) * kTokens;
 
-    // ---- prologue: angles and ring rows of the block's tokens ----
-    for (int i = threadIdx.x; i < kTokens * NP; i += blockDim.x) {
-        const int tl = i / NP, pr = i - tl * NP;
-        const long n = n0 + tl;
-        if (n >= T) continue;
-        const int c = static_cast<int>(n / p.L);
-        const int ic = static_cast<int>(n - static_cast<long>(c) * p.L);
-        const int ax = p.rope.axis[pr];
-        long pos;
-        if (p.pos != nullptr) {
-            pos = __ldg(p.pos + 3 * n + ax);
-        } else {
-            const int hw = p.rope.gh * p.rope.gw;
-            const int f = ic / hw;
-            const int rem = ic - f * hw;
-            const int y = rem / p.rope.gw;
-            pos = ax == 0 ? (p.round + c) * p.rope.F + f : (ax == 1 ? y : rem - y * p.rope.gw);
-        }
-        const double ang = static_cast<double>(pos) * p.rope.omega[pr];
-        const double k = rint(ang * 0.15915494309189535);   // 1 / (2 pi)
-        const float red = static_cast<float>(fma(-k, 6.283185307179586, ang));
-        float sn, cs;
-        sincosf(red, &sn, &cs);
-        s_cs[tl][pr] = make_float2(cs, sn);
-        if (pr == 0) {
-            const int slot = ring_slot(p.round + c, p.R);
-            s_off[tl] = (static_cast<long>(slot) * p.L + ic) * p.H * D;
-        }
-    }
-    __syncthreads();
-
+    // ---- loads first: they do not depend on the angles ----
     const int hl = threadIdx.x / TPR;
     const int part = threadIdx.x - hl * TPR;
     const int h = blockIdx.y * p.heads_per_block + hl;
@@ -120,6 +91,37 @@ __global__ void __launch_bounds__(kMaxThreads) qk_norm_rope_append_kernel(const 
             uq[tl] = uk[tl] = uv[tl] = make_uint4(0u, 0u, 0u, 0u);
         }
     }
+
+    // ---- prologue: angles and ring rows of the block's tokens ----
+    for (int i = threadIdx.x; i < kTokens * NP; i += blockDim.x) {
+        const int tl = i / NP, pr = i - tl * NP;
+        const long n = n0 + tl;
+        if (n >= T) continue;
+        const int c = static_cast<int>(n / p.L);
+        const int ic = static_cast<int>(n - static_cast<long>(c) * p.L);
+        const int ax = p.rope.axis[pr];
+        long pos;
+        if (p.pos != nullptr) {
+            pos = __ldg(p.pos + 3 * n + ax);
+        } else {
+            const int hw = p.rope.gh * p.rope.gw;
+            const int f = ic / hw;
+            const int rem = ic - f * hw;
+            const int y = rem / p.rope.gw;
+            pos = ax == 0 ? (p.round + c) * p.rope.F + f : (ax == 1 ? y : rem - y * p.rope.gw);
+        }
+        const double ang = static_cast<double>(pos) * p.rope.omega[pr];
+        const double k = rint(ang * 0.15915494309189535);   // 1 / (2 pi)
+        const float red = static_cast<float>(fma(-k, 6.283185307179586, ang));
+        float sn, cs;
+        sincosf(red, &sn, &cs);
+        s_cs[tl][pr] = make_float2(cs, sn);
+        if (pr == 0) {
+            const int slot = ring_slot(p.round + c, p.R);
+            s_off[tl] = (static_cast<long>(slot) * p.L + ic) * p.H * D;
+        }
+    }
+    __syncthreads();
 
 #pragma unroll
     for (int tl = 0; tl < kTokens; ++tl) {
