@@ -126,6 +126,13 @@ class ClockSampler:
                     default=None)}
 
 
+def l2_note(working_set_mb):
+    if working_set_mb > 126:
+        return "no flush: per-step working set %.0f MB > 126 MB L2" % working_set_mb
+    return ("no flush: per-step working set %.2f MB fits in L2 (latency-bound workload, "
+            "no roofline claim)" % working_set_mb)
+
+
 def dist_setup(gpus):
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -296,8 +303,7 @@ def run_ours(args, rank, world, local):
             "heads": w.H, "head_dim": w.D, "chunk_tokens": w.L, "wave_chunks": w.n_wave,
             "history_chunks": w.n_hist, "wave_tokens": w.T,
             "parallelism": "replica%d (independent wave rounds, no data-path collective)" % world,
-            "l2": "no flush: per-step working set %.0f MB > 126 MB L2" % (
-                (append_bytes + 2 * w.R * w.L * w.H * w.D * 2) / 1e6),
+            "l2": l2_note((append_bytes + 2 * w.R * w.L * w.H * w.D * 2) / 1e6),
         },
         "chunks_per_s": round(world * w.n_wave / (ms_step * 1e-3), 2),
         "pct_peak": round(100.0 * value / world / peak_tf, 2),
@@ -336,6 +342,132 @@ def run_ours(args, rank, world, local):
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
     return line
+
+
+def run_round_loop(args, rank, world, local):
+    """Full rounds of a multi-layer workload: every round runs, layer after layer,
+    the append and the attention of each layer on that layer's own ring, then
+    advances the ring by one chunk.  Reports per-round latency (median, p90)
+    and rounds/s (one output chunk per round after pipeline fill)."""
+    import torch
+    from chunk_causal_dit_b200 import wf
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = make_group(world, "nccl")
+    w = wi.WORKLOADS[args.workload]
+    peaks, peak_src = load_peaks()
+    plan = wf.Plan(w.L, w.n_wave, w.n_hist, w.H, w.D).set_rope(w.F, w.gh, w.gw)
+    sets = [wi.wave_inputs(w, seed=rank, salt=s) for s in range(2)]   # pool of two input sets
+    qs = [(x.q.to(dev), x.k.to(dev), x.v.to(dev)) for x in sets]
+    gq, gk = sets[0].gamma_q.to(dev), sets[0].gamma_k.to(dev)
+    hk, hv = wi.history_prefill(w, seed=rank)
+    caches = []
+    for _ in range(w.layers):
+        kc = torch.empty((w.R, w.L, w.H, w.D), dtype=torch.bfloat16, device=dev)
+        vc = torch.empty_like(kc)
+        for j in range(w.n_hist):
+            kc[j % w.R].copy_(hk[j])
+            vc[j % w.R].copy_(hv[j])
+        caches.append((kc, vc))
+    q_out = torch.empty_like(qs[0][0])
+    o = torch.empty_like(q_out)
+    stream = torch.cuda.current_stream(dev)
+    r0 = w.n_hist
+    flops_layer = wf.wf_useful_flops(plan, r0)
+
+    def run_round(r, attn_events=None):
+        for layer, (kc, vc) in enumerate(caches):
+            q, k, v = qs[layer % 2]
+            wf.wf_qk_norm_rope_append(plan, r, q, k, v, None, gq, gk, q_out, kc, vc, stream)
+            if attn_events is not None:
+                attn_events[layer][0].record(stream)
+            wf.wf_chunk_causal_attn(plan, r, q_out, kc, vc, o, None, stream)
+            if attn_events is not None:
+                attn_events[layer][1].record(stream)
+
+    rnd = r0
+    for _ in range(args.warmup):
+        run_round(rnd)
+        rnd += 1
+    torch.cuda.synchronize(dev)
+    rounds = args.steps
+    rev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(rounds)]
+    aev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(w.layers)] for _ in range(rounds)]
+    clocks = ClockSampler(local)
+    time.sleep(0.3)
+    barrier(dist, dev)
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    for i in range(rounds):
+        rev[i][0].record(stream)
+        run_round(rnd, aev[i])
+        rev[i][1].record(stream)
+        rnd += 1
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    barrier(dist, dev)
+    clocks.stop()
+    status = wf.wf_sync_status(plan, stream)
+    if status != wf.WF_OK:
+        raise SystemExit("device status %d (%s)" % (status, wf.status_string(status)))
+    per_round = [a.elapsed_time(b) for a, b in rev]
+    total_ms = allreduce_max(dist, sum(per_round), dev)
+    ms_round = total_ms / rounds
+    attn_ms = statistics.mean(a.elapsed_time(b) for rr in aev for a, b in rr)
+    clk = clocks.summary(t_wall0, t_wall1)
+    plan.destroy()
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+    peak_tf = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    attn_tflops = flops_layer / (attn_ms * 1e-3) / 1e12
+    value = aggregate_tflops(world, w.layers * flops_layer, ms_round)
+    srt = sorted(per_round)
+    return {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": rounds,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_round, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded bf16 N(0,1); pool of two q/k/v sets across layers)",
+        "config": {"workload": w.name, "layers": w.layers, "heads": w.H, "head_dim": w.D,
+                   "chunk_tokens": w.L, "wave_chunks": w.n_wave, "history_chunks": w.n_hist,
+                   "step": "one full round: %d x (append + attention), ring advanced" % w.layers,
+                   "parallelism": "replica%d" % world,
+                   "l2": "no flush: per-layer rings total %.1f GB" % (
+                       w.layers * 2 * w.R * w.L * w.H * w.D * 2 / 1e9)},
+        "round_ms_median": round(statistics.median(per_round), 4),
+        "round_ms_p90": round(srt[min(len(srt) - 1, int(0.9 * len(srt)))], 4),
+        "rounds_per_s": round(world * 1e3 / ms_round, 2),
+        "chunks_per_s": round(world * 1e3 / ms_round, 2),
+        "roofline": {
+            "kernel": "chunk_causal_attn_kernel",
+            "bound": "tensor",
+            "achieved": round(attn_tflops, 2),
+            "peak": peak_tf,
+            "unit": "TFLOP/s",
+            "frac": round(attn_tflops / peak_tf, 4),
+            "peak_source": "%s bf16_tflops_sustained (kernel inside a long loop)" % peak_src,
+            "traffic": None,
+            "ms_per_launch": round(attn_ms, 5),
+            "useful_flop_per_launch": flops_layer,
+        },
+        "e2e": None,
+        "e2e_note": "not measured for the multi-layer round (%.1f GB of host q/k/v per round); "
+                    "see the single-layer workload" % (w.layers * 6 * w.T * w.H * w.D / 1e9),
+        "gpu_launches": 2 * w.layers * rounds,
+        "clocks": clk,
+    }
 
 
 # --------------------------------------------------------- oracle (CPU) --
@@ -444,6 +576,8 @@ def main():
     rank, world, local = dist_setup(args.gpus)
     if args.impl == "reference":
         line = run_reference(args, rank, world)
+    elif wi.WORKLOADS[args.workload].layers > 1:
+        line = run_round_loop(args, rank, world, local)
     else:
         line = run_ours(args, rank, world, local)
     if line is not None:

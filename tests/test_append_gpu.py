@@ -95,3 +95,27 @@ def test_append_full_size_wan13b(wf):
     w = wi.WORKLOADS["wan13b_4step"]
     _, ref, out = run_append(wf, w, 2)
     check_append(w, 2, ref, out)
+
+
+def test_append_alternative_tiny_positions(wf):
+    """The tiny wave's description ("t = 0..2, 4x4 grid" with 32-token chunks) also
+    reads as t = chunk index shared by both frames of a chunk; the explicit
+    pos_thw input carries that reading through the same kernel."""
+    w = wi.WORKLOADS["tiny"]
+    x = wi.wave_inputs(w, seed=5)
+    dev = "cuda"
+    n = np.arange(w.T)
+    c, rem = n // w.L, n % w.L
+    pos_np = np.stack([c, (rem % 16) // 4, rem % 4], axis=1).astype(np.int32)
+    plan = wf.Plan(w.L, w.n_wave, w.n_hist, w.H, w.D)      # no geometry: explicit only
+    q_out = torch.empty_like(x.q, device=dev)
+    kc = torch.zeros((w.R, w.L, w.H, w.D), dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros_like(kc)
+    wf.wf_qk_norm_rope_append(plan, 0, x.q.to(dev), x.k.to(dev), x.v.to(dev),
+                              torch.from_numpy(pos_np).to(dev), x.gamma_q.to(dev),
+                              x.gamma_k.to(dev), q_out, kc, vc)
+    torch.cuda.synchronize()
+    ref = oracle.append(wi.bits(x.q), wi.bits(x.k), wi.bits(x.v), pos_np, x.gamma_q.numpy(),
+                        x.gamma_k.numpy(), want_f64=True)
+    check_append(w, 0, ref, (wi.bits(q_out.cpu()), wi.bits(kc.cpu()), wi.bits(vc.cpu())))
+    plan.destroy()
