@@ -421,7 +421,8 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
             if (x == 1 && !un.has1) continue;       // the tile lies past the chunk's end
             const int q_row = (2 * un.pair + x) * BM + row;     // row inside chunk c
             float m_run = -INFINITY, l_run = 0.f;
-            for (int j = 0; j < un.n_kt; ++j) {
+            int t = 0;                              // key tile inside its chunk
+            for (int j = 0; j < un.n_kt; ++j, t = (t + 1 == p.n_ktiles) ? 0 : t + 1) {
                 ok = wait_bar(bar(B::s_full + x), s_phase, ctl, kWhereSoftS);
                 ok = __all_sync(0xFFFFFFFFu, ok);
                 if (!ok) break;
@@ -431,7 +432,6 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tS + q4 * 32, r[q4]);
                 tmem_wait_ld();
-                const int t = j % p.n_ktiles;
                 const int valid = t == p.n_ktiles - 1 ? p.L - t * BN : BN;
                 if (valid < BN) {                   // last tile of a chunk: rows >= L
 #pragma unroll
@@ -440,12 +440,20 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                         for (int e = 0; e < 32; ++e)
                             if (q4 * 32 + e >= valid) r[q4][e] = __float_as_uint(-INFINITY);
                 }
-                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                // row maximum: 8 independent chains of 3-input max, then a tree
+                float mx8[8];
 #pragma unroll
-                for (int k = 0; k < 64; ++k)
-                    mx4[k & 3] = fmax3(mx4[k & 3], __uint_as_float(r[k >> 4][(2 * k) & 31]),
-                                       __uint_as_float(r[k >> 4][(2 * k + 1) & 31]));
-                const float mx = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
+                for (int c = 0; c < 8; ++c)
+                    mx8[c] = fmaxf(__uint_as_float(r[c >> 1][(c & 1) * 16]),
+                                   __uint_as_float(r[c >> 1][(c & 1) * 16 + 1]));
+#pragma unroll
+                for (int k = 1; k < 8; ++k)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        mx8[c] = fmax3(mx8[c], __uint_as_float(r[c >> 1][(c & 1) * 16 + 2 * k]),
+                                       __uint_as_float(r[c >> 1][(c & 1) * 16 + 2 * k + 1]));
+                const float mx = fmaxf(fmax3(mx8[0], mx8[1], mx8[2]),
+                                       fmaxf(fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
                 // The row maximum only moves forward when it grew by more than
                 // 2^8: otherwise exponents stay <= 2^8 against the stale maximum
                 // and O keeps its scale.  (At j = 0 PV overwrites O.)
