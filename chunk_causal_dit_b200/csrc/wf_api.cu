@@ -15,6 +15,8 @@ namespace wf {
 cudaError_t launch_append(const AppendParams &p, int D, cudaStream_t stream);
 cudaError_t launch_attn(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                         const AttnParams &p, int D, int grid, cudaStream_t stream);
+cudaError_t launch_attn_pair(const CUtensorMap &mq, const CUtensorMap &mk64, const CUtensorMap &mv,
+                             const AttnParams &p, cudaStream_t stream);
 }  // namespace wf
 
 namespace {
@@ -52,9 +54,9 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 }
 
 // 4-D map over a [n3][n2][H][D] bf16 tensor (slot/chunk, row, head, channel),
-// box = 64 channels x 1 head x 128 rows x 1 slot, 128-byte swizzle, OOB rows read 0.
+// box = 64 channels x 1 head x box_rows rows x 1 slot, 128-byte swizzle, OOB rows read 0.
 bool encode_map(CUtensorMap *map, const void *base, int D, int H, int n2, int n2_stride_rows,
-                int n3)
+                int n3, int box_rows = 128)
 {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
@@ -63,7 +65,7 @@ bool encode_map(CUtensorMap *map, const void *base, int D, int H, int n2, int n2
     const cuuint64_t row = static_cast<cuuint64_t>(H) * D * 2;
     const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, row,
                                    row * static_cast<cuuint64_t>(n2_stride_rows)};
-    const cuuint32_t box[4] = {64, 1, 128, 1};
+    const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(box_rows), 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -119,6 +121,7 @@ int wf_plan(int chunk_tokens, int n_wave_chunks, int n_hist_chunks, int heads, i
     fill_rope_table(p->rope, p->theta);
     p->wait_limit = kDefaultWaitLimit;
     p->withhold_q = 0;
+    p->attn_kernel = WF_ATTN_AUTO;
     p->device = -1;
     p->num_sms = 0;
     p->cc_major = p->cc_minor = 0;
@@ -191,6 +194,16 @@ int wf_plan_set_withhold_q(wf_plan_t p, int on)
 {
     if (p == nullptr) return WF_ERR_INVALID_ARG;
     p->withhold_q = on ? 1 : 0;
+    return WF_OK;
+}
+
+int wf_plan_set_attn_kernel(wf_plan_t p, int kind)
+{
+    if (p == nullptr) return WF_ERR_INVALID_ARG;
+    if (kind != WF_ATTN_AUTO && kind != WF_ATTN_SINGLE && kind != WF_ATTN_PAIR)
+        return WF_ERR_INVALID_ARG;
+    if (kind == WF_ATTN_PAIR && p->D != 128) return WF_ERR_UNSUPPORTED;
+    p->attn_kernel = kind;
     return WF_OK;
 }
 
@@ -293,8 +306,16 @@ int wf_chunk_causal_attn(wf_plan_t p, long round, const void *q_out, const void 
     a.o = static_cast<uint16_t *>(o);
     a.lse = lse;
     a.words = p->words;
-    const int grid = a.n_units < p->num_sms ? a.n_units : p->num_sms;
-    cudaError_t e = wf::launch_attn(mq, mk, mv, a, p->D, grid, static_cast<cudaStream_t>(stream));
+    const bool pair = p->attn_kernel == WF_ATTN_PAIR;   // AUTO: the single-CTA kernel
+    cudaError_t e;
+    if (pair) {
+        CUtensorMap mk64;
+        if (!encode_map(&mk64, k_cache, p->D, p->H, p->L, p->L, p->R, 64)) return WF_ERR_CUDA;
+        e = wf::launch_attn_pair(mq, mk64, mv, a, static_cast<cudaStream_t>(stream));
+    } else {
+        const int grid = a.n_units < p->num_sms ? a.n_units : p->num_sms;
+        e = wf::launch_attn(mq, mk, mv, a, p->D, grid, static_cast<cudaStream_t>(stream));
+    }
     return e == cudaSuccess ? WF_OK : WF_ERR_CUDA;
 }
 

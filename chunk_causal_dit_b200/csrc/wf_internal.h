@@ -92,6 +92,7 @@ struct wf_plan_s {
     wf::RopeParams rope;
     unsigned long long wait_limit;
     int withhold_q;           // test hook, see wf_plan_set_withhold_q
+    int attn_kernel;          // WF_ATTN_* (wf_plan_set_attn_kernel)
     int device;               // -1: no device state
     int num_sms;
     int cc_major, cc_minor;   // compute capability of `device`

@@ -21,6 +21,11 @@ WF_ERR_TIMEOUT = 4
 WF_ERR_NO_DEVICE = 5
 WF_ERR_DEVICE = 6
 
+# attention kernel variants (wf_plan_set_attn_kernel)
+WF_ATTN_AUTO = 0
+WF_ATTN_SINGLE = 1
+WF_ATTN_PAIR = 2
+
 # Every function include/wf.h declares: name -> (restype, argtypes)
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -32,6 +37,7 @@ SIGNATURES = {
     "wf_plan_set_norm_eps": (_I, [_P, ctypes.c_double]),
     "wf_plan_set_wait_limit": (_I, [_P, ctypes.c_ulonglong]),
     "wf_plan_set_withhold_q": (_I, [_P, _I]),
+    "wf_plan_set_attn_kernel": (_I, [_P, _I]),
     "wf_plan_destroy": (None, [_P]),
     "wf_cache_bytes": (ctypes.c_size_t, [_P]),
     "wf_useful_flops": (ctypes.c_double, [_P, _L]),
@@ -134,6 +140,11 @@ class Plan:
     def set_withhold_q(self, on: bool):
         """Test hook: make the attention kernel's first Q wait expire (see wf.h)."""
         _check(load().wf_plan_set_withhold_q(self.handle, int(bool(on))), "wf_plan_set_withhold_q")
+        return self
+
+    def set_attn_kernel(self, kind: int):
+        """WF_ATTN_AUTO, WF_ATTN_SINGLE or WF_ATTN_PAIR (see wf.h)."""
+        _check(load().wf_plan_set_attn_kernel(self.handle, int(kind)), "wf_plan_set_attn_kernel")
         return self
 
     def destroy(self):

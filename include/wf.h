@@ -93,12 +93,29 @@ WF_API int wf_plan_set_norm_eps(wf_plan_t plan, double eps);
 WF_API int wf_plan_set_wait_limit(wf_plan_t plan, unsigned long long cycles);
 
 /* Test hook for failure detection, off by default.  With on != 0 the attention
- * kernel's producer withholds the first Q-tile copy of every CTA, so the MMA
+ * kernel's producer withholds the first Q-tile copy of every CTA (with the
+ * pair kernel: of every cluster's leader CTA), so the MMA
  * warp's wait for it cannot complete: the bounded wait expires, the kernel
  * stops cleanly (copies and MMAs in flight drained, TMEM freed) and
  * wf_sync_status returns WF_ERR_TIMEOUT.  Nothing faults or traps; the
  * context stays usable.  Pair it with a short wf_plan_set_wait_limit. */
 WF_API int wf_plan_set_withhold_q(wf_plan_t plan, int on);
+
+/* Attention kernel variant.  Both compute the same result (within the
+ * attention tolerance; they accumulate in different orders):
+ *   WF_ATTN_SINGLE  one CTA per SM, two 128-row query tiles per work unit,
+ *                   units taken from a global counter (head_dim 64 and 128);
+ *   WF_ATTN_PAIR    clusters of two CTAs on two SMs sharing 256-row tensor-core
+ *                   MMAs (tcgen05 cta_group::2), S double-buffered in tensor
+ *                   memory, a static longest-first unit order (head_dim 128 only);
+ *   WF_ATTN_AUTO    the default: SINGLE, the faster of the two on B200 at every
+ *                   shape measured (the Wan 1.3B / 14B wave rounds).
+ * Returns WF_ERR_UNSUPPORTED for PAIR with head_dim 64, WF_ERR_INVALID_ARG for
+ * an unknown value. */
+#define WF_ATTN_AUTO 0
+#define WF_ATTN_SINGLE 1
+#define WF_ATTN_PAIR 2
+WF_API int wf_plan_set_attn_kernel(wf_plan_t plan, int kind);
 
 WF_API void wf_plan_destroy(wf_plan_t plan);
 

@@ -67,7 +67,17 @@ def test_plan_setters_validate(wf):
     with pytest.raises(wf.WFError):
         p.set_norm_eps(-1.0)
     p.set_norm_eps(1e-5)
+    for kind in (wf.WF_ATTN_SINGLE, wf.WF_ATTN_PAIR, wf.WF_ATTN_AUTO):
+        p.set_attn_kernel(kind)
+    with pytest.raises(wf.WFError):
+        p.set_attn_kernel(3)
     p.destroy()
+    p64 = wf.Plan(32, 3, 0, 2, 64)
+    p64.set_attn_kernel(wf.WF_ATTN_SINGLE)
+    with pytest.raises(wf.WFError) as e:
+        p64.set_attn_kernel(wf.WF_ATTN_PAIR)   # the pair kernel is head_dim 128 only
+    assert e.value.status == wf.WF_ERR_UNSUPPORTED
+    p64.destroy()
 
 
 @pytest.mark.parametrize("L,W,Hh,H,D", [(32, 3, 0, 2, 64), (4680, 5, 2, 12, 128),

@@ -46,6 +46,14 @@ def oracle_cache_from_ring(kc, vc, round_, W, Hh):
     return cache
 
 
+KERNELS = ["single", "pair"]
+
+
+def make_plan(wf, L, W, Hh, H, D, kernel):
+    kind = {"single": wf.WF_ATTN_SINGLE, "pair": wf.WF_ATTN_PAIR}[kernel]
+    return wf.Plan(L, W, Hh, H, D).set_attn_kernel(kind)
+
+
 def run_attn(wf, plan, round_, q, kc, vc, with_lse=True):
     T, H, D = q.shape
     o = torch.empty_like(q)
@@ -68,10 +76,13 @@ SHAPES = [
 ]
 
 
+@pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("L,W,Hh,H,D,r", SHAPES)
-def test_attention_all_rows(wf, L, W, Hh, H, D, r):
+def test_attention_all_rows(wf, L, W, Hh, H, D, r, kernel):
+    if kernel == "pair" and D != 128:
+        pytest.skip("the pair kernel is built for head_dim 128")
     q, kc, vc = place_round(L, W, Hh, H, D, r, seed=L + W + D)
-    plan = wf.Plan(L, W, Hh, H, D)
+    plan = make_plan(wf, L, W, Hh, H, D, kernel)
     o, lse = run_attn(wf, plan, r, q, kc, vc)
     cache = oracle_cache_from_ring(kc, vc, r, W, Hh)
     T = W * L
@@ -90,10 +101,11 @@ def test_attention_all_rows(wf, L, W, Hh, H, D, r):
     plan.destroy()
 
 
-def test_causality_perturbation_bit_identical(wf):
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_causality_perturbation_bit_identical(wf, kernel):
     L, W, Hh, H, D, r = 200, 4, 2, 2, 128, 6
     q, kc, vc = place_round(L, W, Hh, H, D, r, seed=5)
-    plan = wf.Plan(L, W, Hh, H, D)
+    plan = make_plan(wf, L, W, Hh, H, D, kernel)
     base, _ = run_attn(wf, plan, r, q, kc, vc)
     R = W + Hh
     for j in range(W):
@@ -107,10 +119,11 @@ def test_causality_perturbation_bit_identical(wf):
     plan.destroy()
 
 
-def test_repeat_runs_bit_identical(wf):
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_repeat_runs_bit_identical(wf, kernel):
     L, W, Hh, H, D, r = 4680 // 4, 5, 2, 4, 128, 2
     q, kc, vc = place_round(L, W, Hh, H, D, r, seed=9)
-    plan = wf.Plan(L, W, Hh, H, D)
+    plan = make_plan(wf, L, W, Hh, H, D, kernel)
     first, lse0 = run_attn(wf, plan, r, q, kc, vc)
     for _ in range(5):
         again, lse1 = run_attn(wf, plan, r, q, kc, vc)
@@ -179,9 +192,10 @@ def test_tiny_wave_end_to_end_and_isolated(wf):
     plan.destroy()
 
 
+@pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("name,head_sel", [("wan13b_4step", None), ("wan13b_5step", [0, 5, 11]),
                                            ("wan14b_4step", [0, 1, 22, 39])])
-def test_full_size_sampled(wf, name, head_sel):
+def test_full_size_sampled(wf, name, head_sel, kernel):
     """Full-size round r = n_hist (steady state), the launch the benchmark times;
     checked on rows at chunk and tile boundaries plus random rows."""
     w = wi.WORKLOADS[name]
@@ -189,7 +203,7 @@ def test_full_size_sampled(wf, name, head_sel):
     r = w.n_hist
     x = wi.wave_inputs(w, seed=0)
     hk, hv = wi.history_prefill(w, seed=0)
-    plan = wf.Plan(w.L, w.n_wave, w.n_hist, w.H, w.D).set_rope(w.F, w.gh, w.gw)
+    plan = make_plan(wf, w.L, w.n_wave, w.n_hist, w.H, w.D, kernel).set_rope(w.F, w.gh, w.gw)
     kc = torch.empty((w.R, w.L, w.H, w.D), dtype=torch.bfloat16, device=dev)
     vc = torch.empty_like(kc)
     for j in range(w.n_hist):                 # history chunk ids 0 .. n_hist-1

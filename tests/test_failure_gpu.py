@@ -27,14 +27,15 @@ def wf():
     return mod
 
 
-def test_expired_wait_reports_timeout_and_context_survives(wf):
+@pytest.mark.parametrize("kind", ["WF_ATTN_SINGLE", "WF_ATTN_PAIR"])
+def test_expired_wait_reports_timeout_and_context_survives(wf, kind):
     L, W, Hh, H, D, r = 300, 4, 2, 3, 128, 5
     R = W + Hh
     q = rand_bf16((W * L, H, D), 1)
     kc = rand_bf16((R, L, H, D), 2)
     vc = rand_bf16((R, L, H, D), 3)
     o = torch.empty_like(q)
-    plan = wf.Plan(L, W, Hh, H, D)
+    plan = wf.Plan(L, W, Hh, H, D).set_attn_kernel(getattr(wf, kind))
     plan.set_wait_limit(1 << 24).set_withhold_q(True)    # ~10 ms of SM clock
     wf.wf_chunk_causal_attn(plan, r, q, kc, vc, o, None)
     assert wf.wf_sync_status(plan) == wf.WF_ERR_TIMEOUT
