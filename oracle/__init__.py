@@ -78,6 +78,10 @@ def _load():
         lib.wfo_append.restype = I
         lib.wfo_chunk_causal_attn_rows.argtypes = [I, I, I, P, P, P, P, P, I,
                                                    I, P, P, P, P]
+        lib.wfo_e4m3_encode.argtypes = [P, P, L]
+        lib.wfo_e4m3_decode.argtypes = [P, P, L]
+        lib.wfo_chunk_causal_attn_rows_fp8qk.argtypes = [I, I, I, I, P, P, P, P, P, P, P, I,
+                                                         I, P, P, P, P]
         lib.wfo_chunk_causal_attn_rows.restype = I
         lib.wfo_num_threads.restype = I
         _lib = lib
@@ -230,6 +234,108 @@ def round_attention(cache: OracleCache, round_: int, n_wave: int, n_hist: int,
     k, v, ids = cache.round_keys(round_, n_wave, n_hist)
     qids = np.arange(round_, round_ + n_wave, dtype=np.int64)
     return chunk_causal_attn_rows(q_wave, qids, k, v, ids, cache.L, rows, heads)
+
+
+# ---- FP8 (E4M3) quantized Q.K^T ------------------------------------------------
+
+E4M3_MAX = 448.0
+
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    """E4M3 codes -> float64 values (S.1111.111 decodes to NaN)."""
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    out = np.empty(c.shape, np.float64)
+    _load().wfo_e4m3_decode(_p(c), _p(out), c.size)
+    return out
+
+
+def e4m3_encode(x: np.ndarray) -> np.ndarray:
+    """float64 -> E4M3 codes: round to nearest, ties to even, +-448 saturation."""
+    a = np.ascontiguousarray(x, dtype=np.float64)
+    out = np.empty(a.shape, np.uint8)
+    _load().wfo_e4m3_encode(_p(a), _p(out), a.size)
+    return out
+
+
+def _bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def _fp8_scale(amax: np.ndarray) -> np.ndarray:
+    """Per-group scale in fp32: amax / 448 (IEEE fp32 division), 1 for an all-zero group."""
+    amax = np.asarray(amax, np.float32)
+    return np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+
+
+def _fp8_codes(x32: np.ndarray, scale32: np.ndarray) -> np.ndarray:
+    # the quotient is formed in fp32 (IEEE division), then rounded once to E4M3
+    return e4m3_encode((x32 / scale32).astype(np.float32).astype(np.float64))
+
+
+def quantize_rows_fp8(bits: np.ndarray):
+    """bf16 [N, H, D] -> (E4M3 codes [N, H, D], fp32 scales [H, N]); one scale per
+    (row, head) so that the row's largest magnitude maps to 448."""
+    x = _bf16_bits_to_f32(bits)
+    s = _fp8_scale(np.abs(x).max(axis=2))              # [N, H]
+    return _fp8_codes(x, s[:, :, None]), np.ascontiguousarray(s.T)
+
+
+def quantize_tiles_fp8(bits: np.ndarray, tile: int = 128):
+    """bf16 [L, H, D] of one chunk -> (E4M3 codes [L, H, D], fp32 scales [ceil(L/tile), H]);
+    one scale per (tile of `tile` rows, head)."""
+    x = _bf16_bits_to_f32(bits)
+    L, H, _ = x.shape
+    nt = (L + tile - 1) // tile
+    scales = np.empty((nt, H), np.float32)
+    codes = np.empty(x.shape, np.uint8)
+    for t in range(nt):
+        sl = slice(t * tile, min(L, (t + 1) * tile))
+        scales[t] = _fp8_scale(np.abs(x[sl]).max(axis=(0, 2)))
+        codes[sl] = _fp8_codes(x[sl], scales[t][None, :, None])
+    return codes, scales
+
+
+class OracleCacheFP8:
+    """Absolute chunk id -> (K codes [L,H,D], K scales [nt,H], V bf16 [L,H,D])."""
+
+    def __init__(self, L: int):
+        self.L = L
+        self.chunks: Dict[int, Tuple[np.ndarray, np.ndarray, np.ndarray]] = {}
+
+    def put(self, chunk_id: int, k8: np.ndarray, k_scale: np.ndarray, v: np.ndarray) -> None:
+        self.chunks[int(chunk_id)] = (np.array(k8, np.uint8), np.array(k_scale, np.float32),
+                                      np.array(v, np.uint16))
+
+    def put_bf16(self, chunk_id: int, k_bits: np.ndarray, v_bits: np.ndarray) -> None:
+        """Quantize a bf16 K chunk by the per-tile rule and store it."""
+        k8, ks = quantize_tiles_fp8(k_bits)
+        self.put(chunk_id, k8, ks, v_bits)
+
+
+def round_attention_fp8qk(cache: OracleCacheFP8, round_: int, n_wave: int, n_hist: int,
+                          q8: np.ndarray, q_scale: np.ndarray, rows, heads):
+    """Attention of the given (row, head) pairs of one round with E4M3 q and k
+    (dequantized exactly by their fp32 scales) and bf16 v."""
+    h_valid = min(n_hist, round_)
+    ids = list(range(round_ - h_valid, round_ + n_wave))
+    k8 = np.ascontiguousarray(np.concatenate([cache.chunks[i][0] for i in ids], axis=0))
+    ks = np.ascontiguousarray(np.stack([cache.chunks[i][1] for i in ids], axis=0))
+    v = np.ascontiguousarray(np.concatenate([cache.chunks[i][2] for i in ids], axis=0))
+    kid = np.asarray(ids, np.int64)
+    qid = np.arange(round_, round_ + n_wave, dtype=np.int64)
+    q8 = np.ascontiguousarray(q8, np.uint8)
+    q_scale = np.ascontiguousarray(q_scale, np.float32)
+    rows = np.ascontiguousarray(rows, np.int32)
+    heads = np.ascontiguousarray(heads, np.int32)
+    Tq, H, D = q8.shape
+    o = np.empty((rows.size, D), np.float64)
+    lse = np.empty(rows.size, np.float64)
+    rc = _load().wfo_chunk_causal_attn_rows_fp8qk(H, D, cache.L, Tq, _p(q8), _p(q_scale), _p(qid),
+                                                  _p(k8), _p(ks), _p(v), _p(kid), kid.size,
+                                                  rows.size, _p(rows), _p(heads), _p(o), _p(lse))
+    if rc != 0:
+        raise ValueError("oracle attention: a query row sees no key")
+    return o, lse
 
 
 def useful_flops(L: int, n_wave: int, n_hist: int, H: int, D: int, round_: int) -> float:

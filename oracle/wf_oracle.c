@@ -38,8 +38,22 @@
  *       complete).  s_j = q.k_j / sqrt(D); p = softmax over visible j;
  *       O = sum_j p_j v_j; lse = m + log(sum_j exp(s_j - m)).
  *
- * Parity pins live in tests/test_oracle_pins.py (brute-force dense mask,
- * library softmax attention on the unmasked special case, closed forms and
+ *   wfo_e4m3_encode / wfo_e4m3_decode
+ *       the 8-bit E4M3 floating-point format (1 sign, 4 exponent bits with bias
+ *       7, 3 mantissa bits; exponent field 0 holds subnormals m * 2^-9; no
+ *       infinities; S.1111.111 is NaN; largest finite 1.75 * 2^8 = 448).
+ *       Encoding rounds to nearest, ties to even, and saturates finite values
+ *       beyond 448 to +-448.
+ *
+ *   wfo_chunk_causal_attn_rows_fp8qk
+ *       the same attention with q and k given as E4M3 codes and fp32 scales:
+ *       q~[n,h,:] = e4m3(q8[n,h,:]) * q_scale[h,n] (one scale per row and
+ *       head), k~[j,h,:] = e4m3(k8[j,h,:]) * k_scale[chunk, tile, h] (one scale
+ *       per 128-row key tile of a chunk and head); v stays bf16.
+ *
+ * Parity pins live in tests/test_oracle_pins.py and tests/test_fp8_pins.py
+ * (brute-force dense mask, library softmax attention on the unmasked special
+ * case, the format's published values, a library float8 cast, closed forms and
  * invariants).
  */
 #include <math.h>
@@ -229,6 +243,116 @@ int wfo_chunk_causal_attn_rows(int H, int D, int L,
                 double dot = 0.0;
                 for (int d = 0; d < D; ++d)
                     dot += qd[d] * bf16_bits_to_double(k[(j * H + h) * D + d]);
+                s[j] = dot * scale;
+                if (s[j] > m) m = s[j];
+                ++nvis;
+            }
+            if (nvis == 0) {
+#pragma omp atomic write
+                bad = 1;
+                continue;
+            }
+            double z = 0.0;
+            for (int d = 0; d < D; ++d) acc[d] = 0.0;
+            for (long j = 0; j < nk; ++j) {
+                if (!vis[j]) continue;
+                double w = exp(s[j] - m);
+                z += w;
+                for (int d = 0; d < D; ++d)
+                    acc[d] += w * bf16_bits_to_double(v[(j * H + h) * D + d]);
+            }
+            for (int d = 0; d < D; ++d) o[(long)i * D + d] = acc[d] / z;
+            if (lse) lse[i] = m + log(z);
+        }
+        free(qd); free(s); free(vis); free(acc);
+    }
+    return bad ? -2 : 0;
+}
+
+/* ---- E4M3 ---------------------------------------------------------------- */
+
+static double e4m3_value(uint8_t c)
+{
+    const int sign = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    if (e == 15 && m == 7) return NAN;
+    const double v = e == 0 ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+static uint8_t e4m3_from_double(double x)
+{
+    if (isnan(x)) return 0x7F;
+    const uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    const double a = fabs(x);
+    if (a >= 448.0) return sign | 0x7E;
+    int e;
+    frexp(a, &e);                          /* a = f * 2^e, f in [0.5, 1) */
+    int E = e - 1;                         /* floor(log2 a) */
+    if (a == 0.0 || E < -6) E = -6;        /* subnormal range: quantum 2^-9 */
+    const double quantum = ldexp(1.0, E - 3);
+    const double r = nearbyint(a / quantum);   /* exact quotient, ties to even */
+    const double v = r * quantum;
+    if (v == 0.0) return sign;
+    int e2;
+    frexp(v, &e2);
+    const int E2 = e2 - 1;
+    if (E2 < -6) return sign | (uint8_t)(v / ldexp(1.0, -9));
+    const int mant = (int)(v / ldexp(1.0, E2) * 8.0) - 8;
+    return sign | (uint8_t)((E2 + 7) << 3) | (uint8_t)mant;
+}
+
+void wfo_e4m3_decode(const uint8_t *in, double *out, long n)
+{
+    for (long i = 0; i < n; ++i) out[i] = e4m3_value(in[i]);
+}
+
+void wfo_e4m3_encode(const double *in, uint8_t *out, long n)
+{
+    for (long i = 0; i < n; ++i) out[i] = e4m3_from_double(in[i]);
+}
+
+/*
+ * wfo_chunk_causal_attn_rows_fp8qk: as wfo_chunk_causal_attn_rows, with
+ * q8      : [Tq, H, D] E4M3 codes, q_scale : [H, Tq] fp32
+ * k8      : [n_kchunks*L, H, D] E4M3 codes, k_scale : [n_kchunks, ceil(L/128), H] fp32
+ * v       : [n_kchunks*L, H, D] bf16 bits
+ */
+int wfo_chunk_causal_attn_rows_fp8qk(int H, int D, int L, int Tq,
+                                     const uint8_t *q8, const float *q_scale,
+                                     const int64_t *q_chunk,
+                                     const uint8_t *k8, const float *k_scale,
+                                     const uint16_t *v, const int64_t *k_chunk, int n_kchunks,
+                                     int n_sel, const int32_t *rows, const int32_t *heads,
+                                     double *o, double *lse)
+{
+    const long nk = (long)n_kchunks * L;
+    const int nt = (L + 127) / 128;
+    const double scale = 1.0 / sqrt((double)D);
+    double table[256];
+    for (int c = 0; c < 256; ++c) table[c] = e4m3_value((uint8_t)c);
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *qd = (double *)malloc(sizeof(double) * D);
+        double *s = (double *)malloc(sizeof(double) * (nk > 0 ? nk : 1));
+        unsigned char *vis = (unsigned char *)malloc(nk > 0 ? nk : 1);
+        double *acc = (double *)malloc(sizeof(double) * D);
+#pragma omp for schedule(dynamic, 1)
+        for (int i = 0; i < n_sel; ++i) {
+            const long n = rows[i];
+            const int h = heads[i];
+            const int64_t qid = q_chunk[n / L];
+            const double sq = (double)q_scale[(long)h * Tq + n];
+            for (int d = 0; d < D; ++d) qd[d] = table[q8[(n * H + h) * D + d]] * sq;
+            double m = -INFINITY;
+            long nvis = 0;
+            for (long j = 0; j < nk; ++j) {
+                vis[j] = k_chunk[j / L] <= qid;
+                if (!vis[j]) continue;
+                const long b = j / L, t = (j % L) / 128;
+                const double sk = (double)k_scale[(b * nt + t) * H + h];
+                double dot = 0.0;
+                for (int d = 0; d < D; ++d) dot += qd[d] * (table[k8[(j * H + h) * D + d]] * sk);
                 s[j] = dot * scale;
                 if (s[j] > m) m = s[j];
                 ++nvis;
