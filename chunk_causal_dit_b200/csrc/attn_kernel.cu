@@ -66,14 +66,18 @@ constexpr int kSoftmaxWarpsArrive = 8;      // sched_empty: one arrival per soft
 // MUFU throughput, so the default is 0 (all MUFU); 4 and 8 are tested too.
 constexpr int kEmulatePeriod = 0;
 
-template <int D>
+// F8: Q and K arrive as E4M3 codes (one byte per element, one 128-byte
+// swizzle atom per row at D = 128) with fp32 scales; V, P and O stay as in the
+// bf16 kernel.
+template <int D, bool F8>
 struct Cfg {
     static constexpr int kStages = D == 128 ? 4 : 8;
-    static constexpr int kHalves = D / 64;                 // 128-byte column blocks
+    static constexpr int kHalves = D / 64;                 // 128-byte column blocks (bf16)
     static constexpr uint32_t kHalfBytes = 128 * 128;      // 128 rows x 128 bytes
-    static constexpr uint32_t kTileBytes = BM * D * 2;
+    static constexpr uint32_t kTileBytes = BM * D * 2;     // one bf16 tile = one K/V stage
+    static constexpr uint32_t kQKTileBytes = F8 ? BM * D : kTileBytes;   // a Q or K tile
     static constexpr uint32_t kQOff = 0;
-    static constexpr uint32_t kKVOff = 2 * kTileBytes;
+    static constexpr uint32_t kKVOff = 2 * kQKTileBytes;
     static constexpr uint32_t kBarOff = kKVOff + kStages * kTileBytes;
     static constexpr uint32_t kSmemBytes = kBarOff + 512 + 1024;
     static constexpr uint32_t kS0 = 0, kS1 = 128, kO0 = 256, kO1 = 256 + D;
@@ -144,17 +148,28 @@ __device__ __forceinline__ Unit decode_unit(const AttnParams &p, int u)
 // The descriptors of one operand tile differ only in the start-address field
 // (low 14 bits), so they are built from a 32-bit low word and a constant high
 // word: fewer live 64-bit values in the MMA-issuing thread.
-template <int D>
+template <int D, bool F8>
 __device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t q_smem, uint32_t k_smem)
 {
-    constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, false);
     constexpr uint32_t hi = sw128_desc_hi(1024);
     const uint32_t qlo = sw128_desc_lo(q_smem, 16), klo = sw128_desc_lo(k_smem, 16);
+    if constexpr (F8) {
+        // K = 32 codes (32 bytes) per MMA: four steps along the 128-byte row
+        constexpr uint32_t idesc = idesc_e4m3_f32(BM, BN);
 #pragma unroll
-    for (int s = 0; s < D / 16; ++s) {
-        const uint32_t off = ((s >> 2) * Cfg<D>::kHalfBytes + (s & 3) * 32) >> 4;
-        umma_ss(s_tmem, desc_join(qlo + off, hi), desc_join(klo + off, hi), idesc,
-                s > 0 ? 1u : 0u);
+        for (int s = 0; s < D / 32; ++s) {
+            const uint32_t off = (s * 32) >> 4;
+            umma_ss_f8(s_tmem, desc_join(qlo + off, hi), desc_join(klo + off, hi), idesc,
+                       s > 0 ? 1u : 0u);
+        }
+    } else {
+        constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, false);
+#pragma unroll
+        for (int s = 0; s < D / 16; ++s) {
+            const uint32_t off = ((s >> 2) * Cfg<D, false>::kHalfBytes + (s & 3) * 32) >> 4;
+            umma_ss(s_tmem, desc_join(qlo + off, hi), desc_join(klo + off, hi), idesc,
+                    s > 0 ? 1u : 0u);
+        }
     }
 }
 
@@ -167,7 +182,7 @@ __device__ __forceinline__ void issue_pv_half(uint32_t o_tmem, uint32_t p_tmem, 
     constexpr uint32_t hi = sw128_desc_hi(1024);
     // V tile: 16 keys per step = 2 eight-row groups of 128 bytes; the two
     // 64-channel halves of D sit kHalfBytes apart (leading byte offset).
-    const uint32_t vlo = sw128_desc_lo(v_smem, Cfg<D>::kHalfBytes);
+    const uint32_t vlo = sw128_desc_lo(v_smem, Cfg<D, false>::kHalfBytes);
 #pragma unroll
     for (int i = 0; i < BN / 32; ++i) {
         const int s = half * (BN / 32) + i;
@@ -201,14 +216,14 @@ __device__ __forceinline__ void exp2_fma_pair(float x0, float x1, float &p0, flo
     p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
-template <int D>
+template <int D, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                          const __grid_constant__ CUtensorMap tmap_k,
                          const __grid_constant__ CUtensorMap tmap_v,
                          const AttnParams p)
 {
-    using C = Cfg<D>;
+    using C = Cfg<D, F8>;
     constexpr int S = C::kStages;
     using B = Bars<S>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -281,13 +296,19 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     // thread's bounded wait must expire (tests only)
                     withhold = false;
                 } else {
-                    mbar_arrive_expect_tx(bar(B::q_full), (un.has1 ? 2 : 1) * C::kTileBytes);
+                    mbar_arrive_expect_tx(bar(B::q_full), (un.has1 ? 2 : 1) * C::kQKTileBytes);
                     ++q_fills;
-                    for (int x = 0; x < (un.has1 ? 2 : 1); ++x)
-                        for (int hf = 0; hf < C::kHalves; ++hf)
-                            tma_load_4d(sq + x * C::kTileBytes + hf * C::kHalfBytes, &tmap_q,
-                                        bar(B::q_full), hf * 64, un.h, (2 * un.pair + x) * BM,
-                                        un.c);
+                    for (int x = 0; x < (un.has1 ? 2 : 1); ++x) {
+                        if constexpr (F8) {
+                            tma_load_4d(sq + x * C::kQKTileBytes, &tmap_q, bar(B::q_full), 0,
+                                        un.h, (2 * un.pair + x) * BM, un.c);
+                        } else {
+                            for (int hf = 0; hf < C::kHalves; ++hf)
+                                tma_load_4d(sq + x * C::kQKTileBytes + hf * C::kHalfBytes, &tmap_q,
+                                            bar(B::q_full), hf * 64, un.h, (2 * un.pair + x) * BM,
+                                            un.c);
+                        }
+                    }
                 }
                 for (int j = 0; ok && j < un.n_kt; ++j) {
                     const int b = j / p.n_ktiles;
@@ -297,12 +318,19 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                         if (!(ok = wait_bar(bar(B::kv_empty + stage), kv_phase ^ 1u, ctl,
                                             kWhereProducerKV)))
                             break;
-                        mbar_arrive_expect_tx(bar(B::kv_full + stage), C::kTileBytes);
+                        const bool k_codes = F8 && kv == 0;   // E4M3 K tile: one 128-byte box
+                        mbar_arrive_expect_tx(bar(B::kv_full + stage),
+                                              k_codes ? C::kQKTileBytes : C::kTileBytes);
                         ++kv_fills;
-                        const CUtensorMap *map = kv ? &tmap_v : &tmap_k;
-                        for (int hf = 0; hf < C::kHalves; ++hf)
-                            tma_load_4d(skv + stage * C::kTileBytes + hf * C::kHalfBytes, map,
-                                        bar(B::kv_full + stage), hf * 64, un.h, t * BN, slot);
+                        if (k_codes) {
+                            tma_load_4d(skv + stage * C::kTileBytes, &tmap_k,
+                                        bar(B::kv_full + stage), 0, un.h, t * BN, slot);
+                        } else {
+                            const CUtensorMap *map = kv ? &tmap_v : &tmap_k;
+                            for (int hf = 0; hf < C::kHalves; ++hf)
+                                tma_load_4d(skv + stage * C::kTileBytes + hf * C::kHalfBytes, map,
+                                            bar(B::kv_full + stage), hf * 64, un.h, t * BN, slot);
+                        }
                         if (++stage == S) { stage = 0; kv_phase ^= 1u; }
                     }
                 }
@@ -321,7 +349,7 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
             uint32_t p_phase[2] = {0u, 0u};   // shared by p_half and p_ready (same cadence)
             const uint32_t tS[2] = {tmem + C::kS0, tmem + C::kS1};
             const uint32_t tO[2] = {tmem + C::kO0, tmem + C::kO1};
-            const uint32_t sQ[2] = {sq, sq + C::kTileBytes};
+            const uint32_t sQ[2] = {sq, sq + C::kQKTileBytes};
             bool ok = true;
             // take the next K/V stage in ring order, waiting until its copy landed
 #define WF_NEXT_STAGE(st)                                                              \
@@ -339,10 +367,10 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 q_phase ^= 1u;
                 uint32_t kst;
                 if (!WF_NEXT_STAGE(kst)) break;
-                issue_qk<D>(tS[0], sQ[0], skv + kst * C::kTileBytes);
+                issue_qk<D, F8>(tS[0], sQ[0], skv + kst * C::kTileBytes);
                 umma_commit(bar(B::s_full + 0));
                 if (un.has1) {
-                    issue_qk<D>(tS[1], sQ[1], skv + kst * C::kTileBytes);
+                    issue_qk<D, F8>(tS[1], sQ[1], skv + kst * C::kTileBytes);
                     umma_commit(bar(B::s_full + 1));
                 }
                 umma_commit(bar(B::kv_empty + kst));
@@ -361,7 +389,7 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     issue_pv_half<D>(tO[0], tS[0], skv + vst * C::kTileBytes, 1, true);
                     if (more) {
                         if (!WF_NEXT_STAGE(kst2)) break;
-                        issue_qk<D>(tS[0], sQ[0], skv + kst2 * C::kTileBytes);
+                        issue_qk<D, F8>(tS[0], sQ[0], skv + kst2 * C::kTileBytes);
                         umma_commit(bar(B::s_full + 0));
                     } else {
                         umma_commit(bar(B::o_final + 0));
@@ -381,7 +409,7 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     umma_commit(bar(B::kv_empty + vst));
                     if (more) {
                         if (un.has1) {
-                            issue_qk<D>(tS[1], sQ[1], skv + kst2 * C::kTileBytes);
+                            issue_qk<D, F8>(tS[1], sQ[1], skv + kst2 * C::kTileBytes);
                             umma_commit(bar(B::s_full + 1));
                         }
                         umma_commit(bar(B::kv_empty + kst2));
@@ -404,8 +432,7 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
         const uint32_t lane_sel = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t tS = tmem + lane_sel + (x ? C::kS1 : C::kS0);
         const uint32_t tO = tmem + lane_sel + (x ? C::kO1 : C::kO0);
-        const float scale = p.scale_log2;
-        const uint64_t sc2 = f2_pack(scale, scale);
+        const float scale0 = p.scale_log2;
         uint32_t s_phase = 0, o_phase = 0;
         bool ok = true;
         for (uint32_t it = 0; ok; ++it) {
@@ -420,9 +447,23 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
             const Unit un = decode_unit(p, u);
             if (x == 1 && !un.has1) continue;       // the tile lies past the chunk's end
             const int q_row = (2 * un.pair + x) * BM + row;     // row inside chunk c
+            // F8: the row's Q scale; a key tile's K scale is read per tile below
+            float sq = 1.0f;
+            if constexpr (F8)
+                if (q_row < p.L) sq = p.q_scale[static_cast<long>(un.h) * p.T +
+                                                static_cast<long>(un.c) * p.L + q_row];
             float m_run = -INFINITY, l_run = 0.f;
             int t = 0;                              // key tile inside its chunk
             for (int j = 0; j < un.n_kt; ++j, t = (t + 1 == p.n_ktiles) ? 0 : t + 1) {
+                float scale = scale0;
+                if constexpr (F8) {
+                    // s = (q8 . k8) * sq * sk: fold both scales into the exponent scale
+                    const int b = j / p.n_ktiles;
+                    const int slot = ring_slot(visible_chunk_id(p.round, p.h_valid, b), p.R);
+                    scale = scale0 * sq *
+                            p.k_scale[(static_cast<long>(slot) * p.n_ktiles + t) * p.H + un.h];
+                }
+                const uint64_t sc2 = f2_pack(scale, scale);
                 ok = wait_bar(bar(B::s_full + x), s_phase, ctl, kWhereSoftS);
                 ok = __all_sync(0xFFFFFFFFu, ok);
                 if (!ok) break;
@@ -556,31 +597,39 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
 
 }  // namespace
 
-template <int D>
+template <int D, bool F8>
 static cudaError_t launch_attn_d(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                                  const AttnParams &p, int grid, cudaStream_t stream)
 {
-    const uint32_t smem = Cfg<D>::kSmemBytes;
+    const uint32_t smem = Cfg<D, F8>::kSmemBytes;
     // The setmaxnreg split assumes the kernel was compiled to exactly the
     // launch budget; any other count could leave the increase waiting.
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, chunk_causal_attn_kernel<D>);
+    cudaError_t e = cudaFuncGetAttributes(&fa, chunk_causal_attn_kernel<D, F8>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs != static_cast<int>(kRegsLaunch)) return cudaErrorInvalidKernelImage;
-    e = cudaFuncSetAttribute(chunk_causal_attn_kernel<D>,
+    e = cudaFuncSetAttribute(chunk_causal_attn_kernel<D, F8>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     e = cudaMemsetAsync(&p.words->sched_counter, 0, sizeof(uint32_t), stream);
     if (e != cudaSuccess) return e;
-    chunk_causal_attn_kernel<D><<<grid, kThreads, smem, stream>>>(mq, mk, mv, p);
+    chunk_causal_attn_kernel<D, F8><<<grid, kThreads, smem, stream>>>(mq, mk, mv, p);
     return cudaGetLastError();
 }
 
 cudaError_t launch_attn(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                         const AttnParams &p, int D, int grid, cudaStream_t stream)
 {
-    return D == 128 ? launch_attn_d<128>(mq, mk, mv, p, grid, stream)
-                    : launch_attn_d<64>(mq, mk, mv, p, grid, stream);
+    return D == 128 ? launch_attn_d<128, false>(mq, mk, mv, p, grid, stream)
+                    : launch_attn_d<64, false>(mq, mk, mv, p, grid, stream);
+}
+
+// E4M3 Q and K (maps over the code arrays, box 128 bytes x 1 x 128 rows), bf16 V;
+// head_dim 128 only.
+cudaError_t launch_attn_fp8qk(const CUtensorMap &mq8, const CUtensorMap &mk8, const CUtensorMap &mv,
+                              const AttnParams &p, int grid, cudaStream_t stream)
+{
+    return launch_attn_d<128, true>(mq8, mk8, mv, p, grid, stream);
 }
 
 }  // namespace wf

@@ -164,6 +164,8 @@ extern "C" int wf_chunk_causal_attn_noalloc(int chunk_tokens, int n_wave_chunks,
     a.o = static_cast<uint16_t *>(o);
     a.lse = lse;
     a.words = static_cast<wf::DeviceWords *>(scratch);
+    a.q_scale = nullptr;
+    a.k_scale = nullptr;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // status and timeout site start at zero for this call (the work counter is
     // cleared by the launch itself)

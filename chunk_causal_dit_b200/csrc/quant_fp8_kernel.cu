@@ -1,0 +1,208 @@
+// quant_fp8_kernel.cu -- E4M3 quantization of q_out (one scale per token and head)
+// and of key-cache chunks (one scale per 128-row key tile and head), the inputs of
+// the FP8 Q.K^T attention variant.
+//
+// The quantized Q.K^T is the B200 counterpart of the quantized attention backend
+// the pages run their systems on ("Wave Forcing", abstract: SageAttention with
+// W8A8 backends): scores come from 8-bit operands with per-block fp32 scales,
+// while P.V stays in bf16.
+//
+// Rule (exact, bit-for-bit what the oracle computes): for a group of values x
+// (a row for Q, a key tile for K), amax = max |x| (exact in fp32); the
+// dequantization scale is amax / 448 and the quantization multiplier 448 / amax,
+// both IEEE fp32 divisions (1 when amax = 0); code = E4M3 rounding, ties to
+// even, with saturation, of the IEEE fp32 product x * (448 / amax).
+//
+// Both kernels are HBM-bound: 2 bytes read and 1 byte written per element.
+#include <cuda_bf16.h>
+
+#include "wf_internal.h"
+
+namespace wf {
+
+namespace {
+
+constexpr float kE4M3Max = 448.0f;
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// two E4M3 codes in the low 16 bits: `lo` in bits 0-7, `hi` in bits 8-15
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi)
+{
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+__device__ __forceinline__ float fp8_scale(float amax)
+{
+    return amax > 0.0f ? __fdiv_rn(amax, kE4M3Max) : 1.0f;
+}
+
+__device__ __forceinline__ float fp8_inv(float amax)
+{
+    return amax > 0.0f ? __fdiv_rn(kE4M3Max, amax) : 1.0f;
+}
+
+// 4 codes of x0..x3 * inv, packed little-endian
+__device__ __forceinline__ uint32_t quant4(float x0, float x1, float x2, float x3, float inv)
+{
+    return e4m3x2(__fmul_rn(x0, inv), __fmul_rn(x1, inv)) |
+           (e4m3x2(__fmul_rn(x2, inv), __fmul_rn(x3, inv)) << 16);
+}
+
+__device__ __forceinline__ float warp_max(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+    return v;
+}
+
+// Rows of q [N][H][D] bf16 (row = n * H + h) -> q8 [N][H][D], scale [H][N].
+// A row is D * 2 bytes = D / 8 lanes of 16 bytes; each warp takes 4 loads of
+// 32 / (D / 8) rows, all issued before any reduction.
+template <int D>
+__global__ void __launch_bounds__(256) quantize_rows_kernel(const uint16_t *__restrict__ q,
+                                                            uint8_t *__restrict__ q8,
+                                                            float *__restrict__ scale, long n_rows,
+                                                            int H)
+{
+    constexpr int kLanesPerRow = D / 8;
+    constexpr int kRowsPerLoad = 32 / kLanesPerRow;
+    constexpr int kLoads = 4;
+    constexpr int kRowsPerWarp = kLoads * kRowsPerLoad;
+    const int lane = threadIdx.x & 31;
+    const int sub = lane / kLanesPerRow;              // row within one load
+    const int part = lane % kLanesPerRow;             // 16-byte piece of the row
+    const long row0 = (static_cast<long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * kRowsPerWarp;
+    uint4 w[kLoads];
+#pragma unroll
+    for (int i = 0; i < kLoads; ++i) {
+        const long row = row0 + i * kRowsPerLoad + sub;
+        w[i] = row < n_rows ? __ldcs(reinterpret_cast<const uint4 *>(q + row * D) + part)
+                            : make_uint4(0, 0, 0, 0);
+    }
+    const long n_tok = n_rows / H;
+#pragma unroll
+    for (int i = 0; i < kLoads; ++i) {
+        const long row = row0 + i * kRowsPerLoad + sub;
+        const uint32_t u[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+        float x[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            x[2 * k] = bf16_lo(u[k]);
+            x[2 * k + 1] = bf16_hi(u[k]);
+        }
+        float a = 0.0f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) a = fmaxf(a, fabsf(x[k]));
+#pragma unroll
+        for (int o = kLanesPerRow / 2; o > 0; o >>= 1)
+            a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+        if (row < n_rows) {
+            const float inv = fp8_inv(a);
+            const uint2 c = make_uint2(quant4(x[0], x[1], x[2], x[3], inv),
+                                       quant4(x[4], x[5], x[6], x[7], inv));
+            reinterpret_cast<uint2 *>(q8 + row * D)[part] = c;
+            if (part == 0) {
+                const long n = row / H;
+                const int h = static_cast<int>(row - n * H);
+                scale[static_cast<long>(h) * n_tok + n] = fp8_scale(a);
+            }
+        }
+    }
+}
+
+// One block (8 warps) per (chunk, key tile, head): the tile's rows of one head
+// [R][L][H][D] bf16 -> codes in the same layout, scale [R][n_tiles][H].
+template <int D>
+__global__ void __launch_bounds__(256) quantize_tiles_kernel(const uint16_t *__restrict__ k,
+                                                             uint8_t *__restrict__ k8,
+                                                             float *__restrict__ scale,
+                                                             long first_chunk, int L, int H, int R)
+{
+    constexpr int kPer = D / 32;
+    constexpr int kRowsPerWarp = 16;            // 8 warps x 16 rows = one 128-row tile
+    __shared__ float s_max[8];
+    const int n_tiles = (L + 127) / 128;
+    const int chunk = blockIdx.x / n_tiles;     // index within the quantized range
+    const int t = blockIdx.x - chunk * n_tiles;
+    const int h = blockIdx.y;
+    const int slot = ring_slot(first_chunk + chunk, R);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long slot_base = static_cast<long>(slot) * L;
+
+    float x[kRowsPerWarp][kPer];
+    float a = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kRowsPerWarp; ++i) {
+        const int r = t * 128 + warp + 8 * i;
+        if (r < L) {
+            const uint16_t *src = k + ((slot_base + r) * H + h) * D + lane * kPer;
+            if constexpr (kPer == 4) {
+                const uint2 w = __ldcs(reinterpret_cast<const uint2 *>(src));
+                x[i][0] = bf16_lo(w.x); x[i][1] = bf16_hi(w.x);
+                x[i][2] = bf16_lo(w.y); x[i][3] = bf16_hi(w.y);
+            } else {
+                const uint32_t w = __ldcs(reinterpret_cast<const unsigned int *>(src));
+                x[i][0] = bf16_lo(w); x[i][1] = bf16_hi(w);
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < kPer; ++e) x[i][e] = 0.0f;
+        }
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) a = fmaxf(a, fabsf(x[i][e]));
+    }
+    a = warp_max(a);
+    if (lane == 0) s_max[warp] = a;
+    __syncthreads();
+    a = s_max[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) a = fmaxf(a, s_max[w]);
+    const float inv = fp8_inv(a);
+#pragma unroll
+    for (int i = 0; i < kRowsPerWarp; ++i) {
+        const int r = t * 128 + warp + 8 * i;
+        if (r >= L) continue;
+        uint8_t *dst = k8 + ((slot_base + r) * H + h) * D;
+        if constexpr (kPer == 4) {
+            reinterpret_cast<uint32_t *>(dst)[lane] = quant4(x[i][0], x[i][1], x[i][2], x[i][3], inv);
+        } else {
+            reinterpret_cast<uint16_t *>(dst)[lane] =
+                static_cast<uint16_t>(e4m3x2(__fmul_rn(x[i][0], inv), __fmul_rn(x[i][1], inv)));
+        }
+    }
+    if (threadIdx.x == 0) scale[(static_cast<long>(slot) * n_tiles + t) * H + h] = fp8_scale(a);
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_rows(const uint16_t *q, uint8_t *q8, float *scale, long n_rows, int H,
+                                 int D, cudaStream_t stream)
+{
+    if (n_rows == 0) return cudaSuccess;
+    const long rows_per_block = 8L * 4 * (32 / (D / 8));
+    const dim3 grid(static_cast<unsigned>((n_rows + rows_per_block - 1) / rows_per_block));
+    if (D == 128)
+        quantize_rows_kernel<128><<<grid, 256, 0, stream>>>(q, q8, scale, n_rows, H);
+    else
+        quantize_rows_kernel<64><<<grid, 256, 0, stream>>>(q, q8, scale, n_rows, H);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_tiles(const uint16_t *k, uint8_t *k8, float *scale, long first_chunk,
+                                  int n_chunks, int L, int H, int R, int D, cudaStream_t stream)
+{
+    if (n_chunks == 0) return cudaSuccess;
+    const int n_tiles = (L + 127) / 128;
+    const dim3 grid(static_cast<unsigned>(n_chunks * n_tiles), static_cast<unsigned>(H));
+    if (D == 128)
+        quantize_tiles_kernel<128><<<grid, 256, 0, stream>>>(k, k8, scale, first_chunk, L, H, R);
+    else
+        quantize_tiles_kernel<64><<<grid, 256, 0, stream>>>(k, k8, scale, first_chunk, L, H, R);
+    return cudaGetLastError();
+}
+
+}  // namespace wf

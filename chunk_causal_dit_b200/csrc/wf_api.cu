@@ -17,6 +17,12 @@ cudaError_t launch_attn(const CUtensorMap &mq, const CUtensorMap &mk, const CUte
                         const AttnParams &p, int D, int grid, cudaStream_t stream);
 cudaError_t launch_attn_pair(const CUtensorMap &mq, const CUtensorMap &mk64, const CUtensorMap &mv,
                              const AttnParams &p, cudaStream_t stream);
+cudaError_t launch_attn_fp8qk(const CUtensorMap &mq8, const CUtensorMap &mk8, const CUtensorMap &mv,
+                              const AttnParams &p, int grid, cudaStream_t stream);
+cudaError_t launch_quantize_rows(const uint16_t *q, uint8_t *q8, float *scale, long n_rows, int H,
+                                 int D, cudaStream_t stream);
+cudaError_t launch_quantize_tiles(const uint16_t *k, uint8_t *k8, float *scale, long first_chunk,
+                                  int n_chunks, int L, int H, int R, int D, cudaStream_t stream);
 }  // namespace wf
 
 namespace {
@@ -73,6 +79,28 @@ bool encode_map(CUtensorMap *map, const void *base, int D, int H, int n2, int n2
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
+
+// The same map over a [n3][n2][H][D] array of one-byte E4M3 codes: box = D bytes
+// (one 128-byte swizzle row at D = 128) x 1 head x 128 rows x 1.
+bool encode_map_u8(CUtensorMap *map, const void *base, int D, int H, int n2, int n3)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
+                                static_cast<cuuint64_t>(n2), static_cast<cuuint64_t>(n3)};
+    const cuuint64_t row = static_cast<cuuint64_t>(H) * D;
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D), row,
+                                   row * static_cast<cuuint64_t>(n2)};
+    const cuuint32_t box[4] = {static_cast<cuuint32_t>(D), 1, 128, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void *>(base), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 int check_device(const wf_plan_s *p)
 {
@@ -306,6 +334,8 @@ int wf_chunk_causal_attn(wf_plan_t p, long round, const void *q_out, const void 
     a.o = static_cast<uint16_t *>(o);
     a.lse = lse;
     a.words = p->words;
+    a.q_scale = nullptr;
+    a.k_scale = nullptr;
     const bool pair = p->attn_kernel == WF_ATTN_PAIR;   // AUTO: the single-CTA kernel
     cudaError_t e;
     if (pair) {
@@ -316,6 +346,74 @@ int wf_chunk_causal_attn(wf_plan_t p, long round, const void *q_out, const void 
         const int grid = a.n_units < p->num_sms ? a.n_units : p->num_sms;
         e = wf::launch_attn(mq, mk, mv, a, p->D, grid, static_cast<cudaStream_t>(stream));
     }
+    return e == cudaSuccess ? WF_OK : WF_ERR_CUDA;
+}
+
+int wf_quantize_q_fp8(wf_plan_t p, const void *q_out, void *q8, float *q_scale, void *stream)
+{
+    if (p == nullptr || !q_out || !q8 || !q_scale) return WF_ERR_INVALID_ARG;
+    if (!aligned16(q_out) || !aligned16(q8) || !aligned4(q_scale)) return WF_ERR_INVALID_ARG;
+    if (int s = check_device(p)) return s;
+    const long rows = static_cast<long>(p->L) * p->W * p->H;
+    cudaError_t e = wf::launch_quantize_rows(static_cast<const uint16_t *>(q_out),
+                                             static_cast<uint8_t *>(q8), q_scale, rows, p->H, p->D,
+                                             static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? WF_OK : WF_ERR_CUDA;
+}
+
+int wf_quantize_k_fp8(wf_plan_t p, long first_chunk, int n_chunks, const void *k_cache,
+                      void *k8_cache, float *k_scale, void *stream)
+{
+    if (p == nullptr || first_chunk < 0 || n_chunks < 0 || n_chunks > p->R) return WF_ERR_INVALID_ARG;
+    if (!k_cache || !k8_cache || !k_scale) return WF_ERR_INVALID_ARG;
+    if (!aligned16(k_cache) || !aligned16(k8_cache) || !aligned4(k_scale)) return WF_ERR_INVALID_ARG;
+    if (int s = check_device(p)) return s;
+    cudaError_t e = wf::launch_quantize_tiles(static_cast<const uint16_t *>(k_cache),
+                                              static_cast<uint8_t *>(k8_cache), k_scale, first_chunk,
+                                              n_chunks, p->L, p->H, p->R, p->D,
+                                              static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? WF_OK : WF_ERR_CUDA;
+}
+
+int wf_chunk_causal_attn_fp8qk(wf_plan_t p, long round, const void *q8, const float *q_scale,
+                               const void *k8_cache, const float *k_scale, const void *v_cache,
+                               void *o, float *lse, void *stream)
+{
+    if (p == nullptr || round < 0) return WF_ERR_INVALID_ARG;
+    if (p->D != 128) return WF_ERR_UNSUPPORTED;
+    if (!q8 || !q_scale || !k8_cache || !k_scale || !v_cache || !o) return WF_ERR_INVALID_ARG;
+    if (!aligned16(q8) || !aligned16(k8_cache) || !aligned16(v_cache) || !aligned16(o) ||
+        !aligned4(q_scale) || !aligned4(k_scale) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+        return WF_ERR_INVALID_ARG;
+    if (int s = check_device(p)) return s;
+
+    CUtensorMap mq, mk, mv;
+    if (!encode_map_u8(&mq, q8, p->D, p->H, p->L, p->W) ||
+        !encode_map_u8(&mk, k8_cache, p->D, p->H, p->L, p->R) ||
+        !encode_map(&mv, v_cache, p->D, p->H, p->L, p->L, p->R))
+        return WF_ERR_CUDA;
+
+    wf::AttnParams a;
+    a.round = round;
+    a.L = p->L;
+    a.W = p->W;
+    a.R = p->R;
+    a.H = p->H;
+    a.T = p->L * p->W;
+    a.h_valid = wf::history_valid(round, p->Hh);
+    a.n_ktiles = (p->L + 127) / 128;
+    a.n_qpairs = (a.n_ktiles + 1) / 2;
+    a.n_units = p->H * p->W * a.n_qpairs;
+    a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(p->D)));
+    a.wait_limit = p->wait_limit;
+    a.withhold_q = p->withhold_q;
+    a.o = static_cast<uint16_t *>(o);
+    a.lse = lse;
+    a.words = p->words;
+    a.q_scale = q_scale;
+    a.k_scale = k_scale;
+    const int grid = a.n_units < p->num_sms ? a.n_units : p->num_sms;
+    cudaError_t e = wf::launch_attn_fp8qk(mq, mk, mv, a, grid, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? WF_OK : WF_ERR_CUDA;
 }
 

@@ -81,6 +81,8 @@ struct AttnParams {
     uint16_t *o;
     float *lse;
     DeviceWords *words;
+    const float *q_scale;     // FP8 Q.K^T only: [H][T] per-row Q scales
+    const float *k_scale;     // FP8 Q.K^T only: [R][n_ktiles][H] per-tile K scales
 };
 
 }  // namespace wf

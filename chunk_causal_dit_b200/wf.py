@@ -47,6 +47,9 @@ SIGNATURES = {
     "wf_plan_debug_ranges": (_I, [_P, _L, _P, _I]),
     "wf_status_string": (ctypes.c_char_p, [_I]),
     "wf_chunk_causal_attn_noalloc": (_I, [_I, _I, _I, _I, _I, _L, _P, _P, _P, _P, _P, _P]),
+    "wf_quantize_q_fp8": (_I, [_P, _P, _P, _P, _P]),
+    "wf_quantize_k_fp8": (_I, [_P, _L, _I, _P, _P, _P, _P]),
+    "wf_chunk_causal_attn_fp8qk": (_I, [_P, _L, _P, _P, _P, _P, _P, _P, _P, _P]),
 }
 
 _lib = None
@@ -190,6 +193,29 @@ def wf_chunk_causal_attn(plan: Plan, round_: int, q_out, k_cache, v_cache, o, ls
     _check(load().wf_chunk_causal_attn(plan.handle, round_, _ptr(q_out), _ptr(k_cache),
                                        _ptr(v_cache), _ptr(o), _ptr(lse), _stream(stream)),
            "wf_chunk_causal_attn")
+
+
+def wf_quantize_q_fp8(plan: Plan, q_out, q8, q_scale, stream=None) -> None:
+    """q_out [T,H,D] bf16 -> q8 [T,H,D] uint8 E4M3 codes, q_scale [H,T] float32."""
+    _check(load().wf_quantize_q_fp8(plan.handle, _ptr(q_out), _ptr(q8), _ptr(q_scale),
+                                    _stream(stream)), "wf_quantize_q_fp8")
+
+
+def wf_quantize_k_fp8(plan: Plan, first_chunk: int, n_chunks: int, k_cache, k8_cache, k_scale,
+                      stream=None) -> None:
+    """K of chunks first_chunk.. (ring slots chunk mod R) -> E4M3 codes in k8_cache
+    [R,L,H,D] uint8 and per-tile scales k_scale [R, ceil(L/128), H] float32."""
+    _check(load().wf_quantize_k_fp8(plan.handle, first_chunk, n_chunks, _ptr(k_cache),
+                                    _ptr(k8_cache), _ptr(k_scale), _stream(stream)),
+           "wf_quantize_k_fp8")
+
+
+def wf_chunk_causal_attn_fp8qk(plan: Plan, round_: int, q8, q_scale, k8_cache, k_scale, v_cache,
+                               o, lse=None, stream=None) -> None:
+    _check(load().wf_chunk_causal_attn_fp8qk(plan.handle, round_, _ptr(q8), _ptr(q_scale),
+                                             _ptr(k8_cache), _ptr(k_scale), _ptr(v_cache),
+                                             _ptr(o), _ptr(lse), _stream(stream)),
+           "wf_chunk_causal_attn_fp8qk")
 
 
 def wf_sync_status(plan: Plan, stream=None) -> int:

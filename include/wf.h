@@ -155,6 +155,45 @@ WF_API int wf_chunk_causal_attn(wf_plan_t plan, long round,
                          const void *q_out, const void *k_cache, const void *v_cache,
                          void *o, float *lse, void *stream);
 
+/* ---- FP8 (E4M3) Q.K^T variant --------------------------------------------
+ * The quantized-attention counterpart ("Wave Forcing" abstract: the systems run
+ * on SageAttention with W8A8 backends): Q and K enter the score MMA as 8-bit
+ * E4M3 codes with fp32 scales, P.V stays bf16.  The quantization rule is exact:
+ * for a group x, amax = max|x|, scale = amax / 448 (IEEE fp32 division; 1 for
+ * amax = 0), code = E4M3(x / scale) with the fp32 quotient rounded to nearest,
+ * ties to even, saturating at +-448.  Groups: one (token, head) row of q_out;
+ * one 128-row key tile of one chunk and head of K.  The codes use the layouts of
+ * their bf16 sources with one byte per element. */
+
+/* Quantize q_out [T,H,D] -> q8 [T,H,D] (E4M3 codes) and q_scale [H,T] (fp32),
+ * one scale per (token, head).  Device pointers: q_out and q8 16-byte aligned,
+ * q_scale 4-byte aligned.  One kernel launch on `stream`. */
+WF_API int wf_quantize_q_fp8(wf_plan_t plan, const void *q_out, void *q8, float *q_scale,
+                             void *stream);
+
+/* Quantize the K of absolute chunks first_chunk .. first_chunk+n_chunks-1, read
+ * from k_cache [R,L,H,D] bf16 at slots (chunk mod R), into k8_cache [R,L,H,D]
+ * (E4M3 codes, same slots) and k_scale [R, ceil(L/128), H] (fp32), one scale
+ * per (slot, 128-row key tile, head).  After wf_qk_norm_rope_append(round) the
+ * wave's chunks are first_chunk = round, n_chunks = W; history chunks are
+ * quantized once, when they were appended.  0 <= n_chunks <= R, first_chunk >= 0.
+ * Device pointers as above.  One kernel launch on `stream`. */
+WF_API int wf_quantize_k_fp8(wf_plan_t plan, long first_chunk, int n_chunks,
+                             const void *k_cache, void *k8_cache, float *k_scale,
+                             void *stream);
+
+/* Chunk-causal attention of round r as wf_chunk_causal_attn, with scores
+ * s = (q8 . k8) * q_scale * k_scale / sqrt(D) from an E4M3 tensor-core product
+ * (fp32 accumulation) and bf16 P.V.  head_dim 128 only (WF_ERR_UNSUPPORTED
+ * otherwise).  q8/k8_cache as written by the two calls above; v_cache is the
+ * bf16 ring.  Device pointers (codes and v 16-byte aligned, scales 4-byte
+ * aligned); o must not overlap the inputs.  One persistent kernel launch (plus
+ * a 4-byte memset of the scheduler counter) on `stream`. */
+WF_API int wf_chunk_causal_attn_fp8qk(wf_plan_t plan, long round, const void *q8,
+                                      const float *q_scale, const void *k8_cache,
+                                      const float *k_scale, const void *v_cache, void *o,
+                                      float *lse, void *stream);
+
 /* Wait for `stream`, then read and clear the plan's device status word.
  * Returns WF_OK, WF_ERR_TIMEOUT (a bounded device wait expired) or WF_ERR_CUDA. */
 WF_API int wf_sync_status(wf_plan_t plan, void *stream);

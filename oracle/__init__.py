@@ -262,22 +262,33 @@ def _bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
 
 
 def _fp8_scale(amax: np.ndarray) -> np.ndarray:
-    """Per-group scale in fp32: amax / 448 (IEEE fp32 division), 1 for an all-zero group."""
+    """Per-group dequantization scale in fp32: amax / 448 (IEEE fp32 division), 1 for
+    an all-zero group."""
     amax = np.asarray(amax, np.float32)
     return np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
 
 
-def _fp8_codes(x32: np.ndarray, scale32: np.ndarray) -> np.ndarray:
-    # the quotient is formed in fp32 (IEEE division), then rounded once to E4M3
-    return e4m3_encode((x32 / scale32).astype(np.float32).astype(np.float64))
+def _fp8_inv(amax: np.ndarray) -> np.ndarray:
+    """Per-group quantization multiplier in fp32: 448 / amax (IEEE fp32 division), 1
+    for an all-zero group."""
+    amax = np.asarray(amax, np.float32)
+    safe = np.where(amax > 0, amax, np.float32(1.0)).astype(np.float32)
+    return np.where(amax > 0, np.float32(E4M3_MAX) / safe, np.float32(1.0)).astype(np.float32)
+
+
+def _fp8_codes(x32: np.ndarray, inv32: np.ndarray) -> np.ndarray:
+    # the product is formed in fp32 (IEEE multiply), then rounded once to E4M3
+    return e4m3_encode((x32 * inv32).astype(np.float32).astype(np.float64))
 
 
 def quantize_rows_fp8(bits: np.ndarray):
-    """bf16 [N, H, D] -> (E4M3 codes [N, H, D], fp32 scales [H, N]); one scale per
-    (row, head) so that the row's largest magnitude maps to 448."""
+    """bf16 [N, H, D] -> (E4M3 codes [N, H, D], fp32 scales [H, N]); one group per
+    (row, head): codes = E4M3(x * (448 / amax)), scale = amax / 448, so the group's
+    largest magnitude maps to 448 and code * scale approximates x."""
     x = _bf16_bits_to_f32(bits)
-    s = _fp8_scale(np.abs(x).max(axis=2))              # [N, H]
-    return _fp8_codes(x, s[:, :, None]), np.ascontiguousarray(s.T)
+    amax = np.abs(x).max(axis=2)                       # [N, H]
+    s = _fp8_scale(amax)
+    return _fp8_codes(x, _fp8_inv(amax)[:, :, None]), np.ascontiguousarray(s.T)
 
 
 def quantize_tiles_fp8(bits: np.ndarray, tile: int = 128):
@@ -290,8 +301,9 @@ def quantize_tiles_fp8(bits: np.ndarray, tile: int = 128):
     codes = np.empty(x.shape, np.uint8)
     for t in range(nt):
         sl = slice(t * tile, min(L, (t + 1) * tile))
-        scales[t] = _fp8_scale(np.abs(x[sl]).max(axis=(0, 2)))
-        codes[sl] = _fp8_codes(x[sl], scales[t][None, :, None])
+        amax = np.abs(x[sl]).max(axis=(0, 2))
+        scales[t] = _fp8_scale(amax)
+        codes[sl] = _fp8_codes(x[sl], _fp8_inv(amax)[None, :, None])
     return codes, scales
 
 

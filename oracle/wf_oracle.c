@@ -49,7 +49,8 @@
  *       the same attention with q and k given as E4M3 codes and fp32 scales:
  *       q~[n,h,:] = e4m3(q8[n,h,:]) * q_scale[h,n] (one scale per row and
  *       head), k~[j,h,:] = e4m3(k8[j,h,:]) * k_scale[chunk, tile, h] (one scale
- *       per 128-row key tile of a chunk and head); v stays bf16.
+ *       per 128-row key tile of a chunk and head); v stays bf16.  (The codes
+ *       and scales come from the quantization rule in oracle/__init__.py.)
  *
  * Parity pins live in tests/test_oracle_pins.py and tests/test_fp8_pins.py
  * (brute-force dense mask, library softmax attention on the unmasked special

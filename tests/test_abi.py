@@ -28,7 +28,7 @@ def wf():
 def header_functions():
     text = open(os.path.join(ROOT, "include", "wf.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(wf_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(wf_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_library_exports_every_declared_symbol(wf):
