@@ -202,10 +202,28 @@ def run_ours(args, rank, world, local):
     flops_step = wf.wf_useful_flops(plan, r0)
     tensor_bytes = w.T * w.H * w.D * 2
     append_bytes = 12 * w.T * w.H * w.D
+    fp8 = args.attn == "fp8qk"
+    if fp8:
+        # E4M3 copies of q_out (per row) and of the key ring (per 128-row tile);
+        # the history chunks were quantized when they were appended
+        nt = (w.L + 127) // 128
+        q8 = torch.empty((w.T, w.H, w.D), dtype=torch.uint8, device=dev)
+        q_scale = torch.empty((w.H, w.T), dtype=torch.float32, device=dev)
+        k8 = torch.empty((w.R, w.L, w.H, w.D), dtype=torch.uint8, device=dev)
+        k_scale = torch.empty((w.R, nt, w.H), dtype=torch.float32, device=dev)
+        wf.wf_quantize_k_fp8(plan, 0, w.n_hist, kc, k8, k_scale, stream)
+
+    def attention(r):
+        if fp8:
+            wf.wf_quantize_q_fp8(plan, q_out, q8, q_scale, stream)
+            wf.wf_quantize_k_fp8(plan, r, w.n_wave, kc, k8, k_scale, stream)
+            wf.wf_chunk_causal_attn_fp8qk(plan, r, q8, q_scale, k8, k_scale, vc, o, None, stream)
+        else:
+            wf.wf_chunk_causal_attn(plan, r, q_out, kc, vc, o, None, stream)
 
     def step(r):
         wf.wf_qk_norm_rope_append(plan, r, q, k, v, None, gq, gk, q_out, kc, vc, stream)
-        wf.wf_chunk_causal_attn(plan, r, q_out, kc, vc, o, None, stream)
+        attention(r)
 
     rnd = r0
     for _ in range(args.warmup):
@@ -217,7 +235,8 @@ def run_ours(args, rank, world, local):
 
     # ---- device-timed steps (kernel events inside give the roofline) ----
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+           torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
     time.sleep(0.3)
@@ -226,11 +245,19 @@ def run_ours(args, rank, world, local):
     t_wall0 = time.time()
     start.record(stream)
     for i in range(args.steps):
-        e0, e1, e2 = ev[i]
+        e0, e1, eq, e2 = ev[i]
         e0.record(stream)
         wf.wf_qk_norm_rope_append(plan, rnd, q, k, v, None, gq, gk, q_out, kc, vc, stream)
         e1.record(stream)
-        wf.wf_chunk_causal_attn(plan, rnd, q_out, kc, vc, o, None, stream)
+        if fp8:
+            wf.wf_quantize_q_fp8(plan, q_out, q8, q_scale, stream)
+            wf.wf_quantize_k_fp8(plan, rnd, w.n_wave, kc, k8, k_scale, stream)
+            eq.record(stream)
+            wf.wf_chunk_causal_attn_fp8qk(plan, rnd, q8, q_scale, k8, k_scale, vc, o, None,
+                                          stream)
+        else:
+            eq.record(stream)
+            wf.wf_chunk_causal_attn(plan, rnd, q_out, kc, vc, o, None, stream)
         e2.record(stream)
         rnd += 1
     stop.record(stream)
@@ -243,10 +270,12 @@ def run_ours(args, rank, world, local):
         raise SystemExit("device status %d (%s)" % (status, wf.status_string(status)))
     ms_total = allreduce_max(dist, start.elapsed_time(stop), dev)
     ms_step = ms_total / args.steps
-    t_append = [a.elapsed_time(b) for a, b, _ in ev]
-    t_attn = [b.elapsed_time(c) for _, b, c in ev]
+    t_append = [a.elapsed_time(b) for a, b, _, _ in ev]
+    t_quant = [b.elapsed_time(c) for _, b, c, _ in ev]
+    t_attn = [c.elapsed_time(d) for _, _, c, d in ev]
     attn_ms = statistics.mean(t_attn)
     append_ms = statistics.mean(t_append)
+    quant_ms = statistics.mean(t_quant)
 
     # ---- end to end through the API: pinned host in, pinned host out ----
     # Every round copies its q, k, v from pinned host memory and its O back;
@@ -258,7 +287,8 @@ def run_ours(args, rank, world, local):
     hv_ = x.v.pin_memory()
     ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
     e2e_steps = max(3, min(args.steps, 50))
-    pipe = HostRoundPipeline(plan, kc, vc, gq, gk, device=dev)
+    pipe = HostRoundPipeline(plan, kc, vc, gq, gk, device=dev,
+                             fp8=(k8, k_scale) if fp8 else None)
     pipe.run([(rnd + i, hq, hk_, hv_, ho) for i in range(2)])
     rnd += 2
     pipe.synchronize()
@@ -281,6 +311,14 @@ def run_ours(args, rank, world, local):
         return None
 
     peak_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    peak_src_note = "%s bf16_tflops (burst)" % peak_src
+    if fp8:
+        # half the useful FLOPs (Q.K^T) run on E4M3 at twice the bf16 rate
+        # (nominal 4.5 vs 2.25 PF dense), half (P.V) on bf16: the contraction's
+        # peak is 1 / (0.5 / 2 + 0.5) = 4/3 of the measured bf16 peak
+        peak_tf = round(peak_tf * 4.0 / 3.0, 1)
+        peak_src_note = ("4/3 x %s bf16_tflops (burst): Q.K^T at the nominal 2x E4M3 rate, "
+                         "P.V at bf16" % peak_src)
     attn_tflops = flops_step / (attn_ms * 1e-3) / 1e12
     value = aggregate_tflops(world, flops_step, ms_step)
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
@@ -296,26 +334,26 @@ def run_ours(args, rank, world, local):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "e4m3 q.k^t, bf16 p.v" if fp8 else "bf16",
         "data": "synthetic (seeded bf16 N(0,1) q/k/v and history, gains 1+0.1N(0,1))",
         "config": {
             "workload": w.name,
             "heads": w.H, "head_dim": w.D, "chunk_tokens": w.L, "wave_chunks": w.n_wave,
-            "history_chunks": w.n_hist, "wave_tokens": w.T,
+            "history_chunks": w.n_hist, "wave_tokens": w.T, "attention": args.attn,
             "parallelism": "replica%d (independent wave rounds, no data-path collective)" % world,
             "l2": l2_note((append_bytes + 2 * w.R * w.L * w.H * w.D * 2) / 1e6),
         },
         "chunks_per_s": round(world * w.n_wave / (ms_step * 1e-3), 2),
         "pct_peak": round(100.0 * value / world / peak_tf, 2),
         "roofline": {
-            "kernel": "chunk_causal_attn_kernel",
+            "kernel": "chunk_causal_attn_kernel<128, fp8>" if fp8 else "chunk_causal_attn_kernel",
             "bound": "tensor",
             "achieved": round(attn_tflops, 2),
             "peak": peak_tf,
             "unit": "TFLOP/s",
             "frac": round(attn_tflops / peak_tf, 4),
-            "peak_source": "%s bf16_tflops (burst)" % peak_src,
-            "traffic": profiled_traffic(args.workload),
+            "peak_source": peak_src_note,
+            "traffic": profiled_traffic(args.workload + ("/fp8qk" if fp8 else "")),
             "ms_per_launch": round(attn_ms, 5),
             "useful_flop_per_launch": flops_step,
         },
@@ -329,6 +367,16 @@ def run_ours(args, rank, world, local):
             "frac": round(append_gbs / hbm, 4),
             "bytes_per_launch": append_bytes,
         },
+        **({"quantize": {
+            "kernels": "quantize_rows_kernel + quantize_tiles_kernel (wave chunks)",
+            "bound": "hbm",
+            "ms_per_step": round(quant_ms, 5),
+            "achieved": round(6 * w.T * w.H * w.D / (quant_ms * 1e-3) / 1e9, 1),
+            "peak": hbm,
+            "unit": "GB/s",
+            "frac": round(6 * w.T * w.H * w.D / (quant_ms * 1e-3) / 1e9 / hbm, 4),
+            "bytes_per_step": 6 * w.T * w.H * w.D,
+        }} if fp8 else {}),
         "e2e": {
             "value": round(aggregate_tflops(world, flops_step, e2e_ms), 3),
             "unit": "TFLOP/s",
@@ -336,7 +384,7 @@ def run_ours(args, rank, world, local):
             "h2d_bytes_per_step": 3 * tensor_bytes,
             "d2h_bytes_per_step": tensor_bytes,
         },
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": (5 if fp8 else 2) * args.steps,
         "clocks": clk,
     }
     if not args.no_cpu_baseline and world == 1:
@@ -568,11 +616,15 @@ def main():
     ap.add_argument("--workload", default="wan13b_4step", choices=sorted(wi.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--attn", default="bf16", choices=["bf16", "fp8qk"],
+                    help="attention variant: bf16 (default) or E4M3 Q.K^T with bf16 P.V")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--ref-pairs", type=int, default=48)
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    if args.attn != "bf16" and wi.WORKLOADS[args.workload].layers > 1:
+        raise SystemExit("--attn %s times single-layer workloads only" % args.attn)
     rank, world, local = dist_setup(args.gpus)
     if args.impl == "reference":
         line = run_reference(args, rank, world)

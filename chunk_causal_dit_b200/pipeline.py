@@ -8,7 +8,9 @@ the binding in ``chunk_causal_dit_b200.wf``.
 
 Per round i (staging slot s = i % 2):
   copy-in stream : q, k, v host -> device slot s   (after round i-2 released s)
-  compute stream : wf_qk_norm_rope_append, wf_chunk_causal_attn (after copy-in)
+  compute stream : wf_qk_norm_rope_append, wf_chunk_causal_attn (after copy-in);
+                   with the FP8 Q.K^T variant: append, wf_quantize_q_fp8,
+                   wf_quantize_k_fp8 of the wave's chunks, wf_chunk_causal_attn_fp8qk
   copy-out stream: O device slot s -> host         (after the attention)
 """
 from __future__ import annotations
@@ -25,11 +27,14 @@ class HostRoundPipeline:
 
     plan, k_cache, v_cache, gamma_q, gamma_k: as for the direct calls (device
     tensors).  pos_thw: optional device tensor [T, 3] (None = derived positions).
+    fp8: optional (k8_cache, k_scale) device tensors; when given, every round runs
+    the FP8 Q.K^T variant and keeps the E4M3 key ring up to date.
     """
 
     def __init__(self, plan: "wf.Plan", k_cache, v_cache, gamma_q, gamma_k,
-                 pos_thw=None, device: Optional[torch.device] = None):
+                 pos_thw=None, device: Optional[torch.device] = None, fp8=None):
         self.plan = plan
+        self.fp8 = fp8
         self.kc, self.vc = k_cache, v_cache
         self.gq, self.gk = gamma_q, gamma_k
         self.pos = pos_thw
@@ -41,6 +46,9 @@ class HostRoundPipeline:
         self.v = [torch.empty(shape, dtype=bf, device=self.dev) for _ in range(2)]
         self.q_out = torch.empty(shape, dtype=bf, device=self.dev)
         self.o = [torch.empty(shape, dtype=bf, device=self.dev) for _ in range(2)]
+        if fp8 is not None:
+            self.q8 = torch.empty(shape, dtype=torch.uint8, device=self.dev)
+            self.q_scale = torch.empty((plan.H, plan.T), dtype=torch.float32, device=self.dev)
         self.s_in = torch.cuda.Stream(self.dev)
         self.s_out = torch.cuda.Stream(self.dev)
         self.s_comp = torch.cuda.Stream(self.dev)
@@ -87,8 +95,15 @@ class HostRoundPipeline:
                                       self.pos, self.gq, self.gk, self.q_out, self.kc, self.vc,
                                       c)
             self.in_free[slot].record(c)
-            wf.wf_chunk_causal_attn(self.plan, r, self.q_out, self.kc, self.vc, self.o[slot],
-                                    None, c)
+            if self.fp8 is None:
+                wf.wf_chunk_causal_attn(self.plan, r, self.q_out, self.kc, self.vc,
+                                        self.o[slot], None, c)
+            else:
+                k8, ks = self.fp8
+                wf.wf_quantize_q_fp8(self.plan, self.q_out, self.q8, self.q_scale, c)
+                wf.wf_quantize_k_fp8(self.plan, r, self.plan.W, self.kc, k8, ks, c)
+                wf.wf_chunk_causal_attn_fp8qk(self.plan, r, self.q8, self.q_scale, k8, ks,
+                                              self.vc, self.o[slot], None, c)
             self.o_ready[slot].record(c)
             with torch.cuda.stream(self.s_out):
                 self.s_out.wait_event(self.o_ready[slot])
