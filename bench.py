@@ -38,6 +38,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 BAD_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
 
 
+# nominal dense bf16 tensor peak and HBM3e bandwidth of one B200 (for the second
+# fraction next to the measured-peak one)
+NOMINAL_BF16_TFLOPS = 2250.0
+NOMINAL_HBM_GBS = 8000.0
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -343,7 +349,9 @@ def run_ours(args, rank, world, local):
             "parallelism": "replica%d (independent wave rounds, no data-path collective)" % world,
             "l2": l2_note((append_bytes + 2 * w.R * w.L * w.H * w.D * 2) / 1e6),
         },
-        "chunks_per_s": round(world * w.n_wave / (ms_step * 1e-3), 2),
+        # query chunks per second of attention (W / t_attn) and of the whole step
+        "chunks_per_s": round(world * w.n_wave / (attn_ms * 1e-3), 2),
+        "chunks_per_s_step": round(world * w.n_wave / (ms_step * 1e-3), 2),
         "pct_peak": round(100.0 * value / world / peak_tf, 2),
         "roofline": {
             "kernel": "chunk_causal_attn_kernel<128, fp8>" if fp8 else "chunk_causal_attn_kernel",
@@ -352,6 +360,8 @@ def run_ours(args, rank, world, local):
             "peak": peak_tf,
             "unit": "TFLOP/s",
             "frac": round(attn_tflops / peak_tf, 4),
+            "frac_nominal": round(attn_tflops / (NOMINAL_BF16_TFLOPS * (4.0 / 3.0 if fp8 else 1.0)),
+                                  4),
             "peak_source": peak_src_note,
             "traffic": profiled_traffic(args.workload + ("/fp8qk" if fp8 else "")),
             "ms_per_launch": round(attn_ms, 5),
@@ -365,6 +375,7 @@ def run_ours(args, rank, world, local):
             "peak": hbm,
             "unit": "GB/s",
             "frac": round(append_gbs / hbm, 4),
+            "frac_nominal": round(append_gbs / NOMINAL_HBM_GBS, 4),
             "bytes_per_launch": append_bytes,
         },
         **({"quantize": {

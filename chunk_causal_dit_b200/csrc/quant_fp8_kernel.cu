@@ -115,15 +115,19 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const uint16_t *__re
 }
 
 // One block (8 warps) per (chunk, key tile, head): the tile's rows of one head
-// [R][L][H][D] bf16 -> codes in the same layout, scale [R][n_tiles][H].
+// [R][L][H][D] bf16 -> codes in the same layout, scale [R][n_tiles][H].  A row is
+// D / 8 lanes of 16 bytes; each warp loads 128 / 8 = 16 rows in kLoads loads of
+// 32 / (D / 8) rows and keeps them in registers between the amax and the
+// quantize passes.
 template <int D>
 __global__ void __launch_bounds__(256) quantize_tiles_kernel(const uint16_t *__restrict__ k,
                                                              uint8_t *__restrict__ k8,
                                                              float *__restrict__ scale,
                                                              long first_chunk, int L, int H, int R)
 {
-    constexpr int kPer = D / 32;
-    constexpr int kRowsPerWarp = 16;            // 8 warps x 16 rows = one 128-row tile
+    constexpr int kLanesPerRow = D / 8;
+    constexpr int kRowsPerLoad = 32 / kLanesPerRow;
+    constexpr int kLoads = 16 / kRowsPerLoad;   // 16 rows per warp, 8 warps = 128 rows
     __shared__ float s_max[8];
     const int n_tiles = (L + 127) / 128;
     const int chunk = blockIdx.x / n_tiles;     // index within the quantized range
@@ -131,48 +135,41 @@ __global__ void __launch_bounds__(256) quantize_tiles_kernel(const uint16_t *__r
     const int h = blockIdx.y;
     const int slot = ring_slot(first_chunk + chunk, R);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int sub = lane / kLanesPerRow, part = lane % kLanesPerRow;
     const long slot_base = static_cast<long>(slot) * L;
+    const int row_base = t * 128 + warp * 16;
 
-    float x[kRowsPerWarp][kPer];
+    uint4 w[kLoads];
+#pragma unroll
+    for (int i = 0; i < kLoads; ++i) {
+        const int r = row_base + i * kRowsPerLoad + sub;
+        w[i] = r < L ? __ldcs(reinterpret_cast<const uint4 *>(k + ((slot_base + r) * H + h) * D) +
+                              part)
+                     : make_uint4(0, 0, 0, 0);
+    }
     float a = 0.0f;
 #pragma unroll
-    for (int i = 0; i < kRowsPerWarp; ++i) {
-        const int r = t * 128 + warp + 8 * i;
-        if (r < L) {
-            const uint16_t *src = k + ((slot_base + r) * H + h) * D + lane * kPer;
-            if constexpr (kPer == 4) {
-                const uint2 w = __ldcs(reinterpret_cast<const uint2 *>(src));
-                x[i][0] = bf16_lo(w.x); x[i][1] = bf16_hi(w.x);
-                x[i][2] = bf16_lo(w.y); x[i][3] = bf16_hi(w.y);
-            } else {
-                const uint32_t w = __ldcs(reinterpret_cast<const unsigned int *>(src));
-                x[i][0] = bf16_lo(w); x[i][1] = bf16_hi(w);
-            }
-        } else {
+    for (int i = 0; i < kLoads; ++i) {
+        const uint32_t u[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
 #pragma unroll
-            for (int e = 0; e < kPer; ++e) x[i][e] = 0.0f;
-        }
-#pragma unroll
-        for (int e = 0; e < kPer; ++e) a = fmaxf(a, fabsf(x[i][e]));
+        for (int e = 0; e < 4; ++e) a = fmaxf(a, fmaxf(fabsf(bf16_lo(u[e])), fabsf(bf16_hi(u[e]))));
     }
     a = warp_max(a);
     if (lane == 0) s_max[warp] = a;
     __syncthreads();
     a = s_max[0];
 #pragma unroll
-    for (int w = 1; w < 8; ++w) a = fmaxf(a, s_max[w]);
+    for (int v = 1; v < 8; ++v) a = fmaxf(a, s_max[v]);
     const float inv = fp8_inv(a);
 #pragma unroll
-    for (int i = 0; i < kRowsPerWarp; ++i) {
-        const int r = t * 128 + warp + 8 * i;
+    for (int i = 0; i < kLoads; ++i) {
+        const int r = row_base + i * kRowsPerLoad + sub;
         if (r >= L) continue;
-        uint8_t *dst = k8 + ((slot_base + r) * H + h) * D;
-        if constexpr (kPer == 4) {
-            reinterpret_cast<uint32_t *>(dst)[lane] = quant4(x[i][0], x[i][1], x[i][2], x[i][3], inv);
-        } else {
-            reinterpret_cast<uint16_t *>(dst)[lane] =
-                static_cast<uint16_t>(e4m3x2(__fmul_rn(x[i][0], inv), __fmul_rn(x[i][1], inv)));
-        }
+        const uint32_t u[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+        const uint2 c = make_uint2(
+            quant4(bf16_lo(u[0]), bf16_hi(u[0]), bf16_lo(u[1]), bf16_hi(u[1]), inv),
+            quant4(bf16_lo(u[2]), bf16_hi(u[2]), bf16_lo(u[3]), bf16_hi(u[3]), inv));
+        reinterpret_cast<uint2 *>(k8 + ((slot_base + r) * H + h) * D)[part] = c;
     }
     if (threadIdx.x == 0) scale[(static_cast<long>(slot) * n_tiles + t) * H + h] = fp8_scale(a);
 }

@@ -143,6 +143,37 @@ def test_hot_calls_without_device(wf):
     p.destroy()
 
 
+def test_fp8_calls_validate_before_the_device(wf):
+    """The FP8 entry points: argument checks (NULL, alignment, chunk range,
+    head_dim) come before any device access; with valid arguments and no GPU the
+    calls report WF_ERR_NO_DEVICE."""
+    import torch
+    lib = wf.load()
+    fake = 1 << 20
+    p = wf.Plan(300, 4, 2, 3, 128)
+    # head_dim 64 is unsupported by the FP8 attention, whatever the pointers
+    p64 = wf.Plan(32, 3, 0, 2, 64)
+    assert lib.wf_chunk_causal_attn_fp8qk(p64.handle, 0, fake, fake, fake, fake, fake, fake,
+                                          None, None) == wf.WF_ERR_UNSUPPORTED
+    assert lib.wf_chunk_causal_attn_fp8qk(p.handle, 0, None, fake, fake, fake, fake, fake,
+                                          None, None) == wf.WF_ERR_INVALID_ARG
+    assert lib.wf_chunk_causal_attn_fp8qk(p.handle, 0, fake + 8, fake, fake, fake, fake, fake,
+                                          None, None) == wf.WF_ERR_INVALID_ARG
+    assert lib.wf_chunk_causal_attn_fp8qk(p.handle, 0, fake, fake + 2, fake, fake, fake, fake,
+                                          None, None) == wf.WF_ERR_INVALID_ARG
+    assert lib.wf_quantize_q_fp8(p.handle, fake, fake + 4, fake, None) == wf.WF_ERR_INVALID_ARG
+    assert lib.wf_quantize_k_fp8(p.handle, 0, 7, fake, fake, fake, None) == wf.WF_ERR_INVALID_ARG
+    assert lib.wf_quantize_k_fp8(p.handle, -1, 1, fake, fake, fake, None) == wf.WF_ERR_INVALID_ARG
+    if not torch.cuda.is_available():
+        assert lib.wf_quantize_q_fp8(p.handle, fake, fake, fake, None) == wf.WF_ERR_NO_DEVICE
+        assert lib.wf_quantize_k_fp8(p.handle, 3, 6, fake, fake, fake, None) == \
+            wf.WF_ERR_NO_DEVICE
+        assert lib.wf_chunk_causal_attn_fp8qk(p.handle, 0, fake, fake, fake, fake, fake, fake,
+                                              None, None) == wf.WF_ERR_NO_DEVICE
+    p.destroy()
+    p64.destroy()
+
+
 def test_status_strings(wf):
     assert wf.status_string(0) == "ok"
     assert "timed out" in wf.status_string(wf.WF_ERR_TIMEOUT)
