@@ -102,6 +102,31 @@ def test_attention_all_rows(wf, L, W, Hh, H, D, r, kernel):
 
 
 @pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("L,H,D", [(300, 2, 128), (700, 1, 128), (200, 3, 64)])
+def test_single_chunk_equals_bidirectional_attention(wf, L, H, D, kernel):
+    """One wave chunk and no history: chunk-causal attention is plain
+    bidirectional softmax attention over the chunk.  Checked against PyTorch's
+    scaled_dot_product_attention in fp64 on the same bf16 values (a library
+    route independent of the oracle) and against the oracle."""
+    if kernel == "pair" and D != 128:
+        pytest.skip("the pair kernel is built for head_dim 128")
+    q, kc, vc = place_round(L, 1, 0, H, D, 0, seed=L + 7 * H)
+    plan = make_plan(wf, L, 1, 0, H, D, kernel)
+    o, lse = run_attn(wf, plan, 0, q, kc, vc)
+    qd = q.cpu().double().permute(1, 0, 2)            # [H, L, D]
+    kd = kc[0].cpu().double().permute(1, 0, 2)
+    vd = vc[0].cpu().double().permute(1, 0, 2)
+    ref = torch.nn.functional.scaled_dot_product_attention(qd[None], kd[None], vd[None])[0]
+    ref = ref.permute(1, 0, 2).reshape(L * H, D).numpy()
+    got = o.float().cpu().numpy().reshape(L * H, D)
+    assert_attention_close(got, ref, "single chunk vs sdpa L=%d D=%d" % (L, D))
+    s_ = torch.einsum("hld,hmd->hlm", qd, kd) / np.sqrt(D)
+    lse_ref = torch.logsumexp(s_, dim=-1).numpy()     # [H, L]
+    assert np.max(np.abs(lse.cpu().numpy() - lse_ref)) <= 1e-3
+    plan.destroy()
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
 def test_causality_perturbation_bit_identical(wf, kernel):
     L, W, Hh, H, D, r = 200, 4, 2, 2, 128, 6
     q, kc, vc = place_round(L, W, Hh, H, D, r, seed=5)

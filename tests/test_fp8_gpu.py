@@ -88,6 +88,7 @@ SHAPES = [
     (129, 3, 3, 2, 1),      # one row past a tile, pipeline filling
     (513, 2, 2, 1, 9),      # odd number of query tiles
     (128, 2, 0, 1, 0),      # one tile, no history
+    (300, 1, 0, 2, 0),      # a single chunk: plain bidirectional attention
 ]
 
 
