@@ -127,6 +127,53 @@ def test_single_chunk_equals_bidirectional_attention(wf, L, H, D, kernel):
 
 
 @pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("D", [128, 64])
+def test_score_jump_far_above_the_running_reference(wf, D, kernel):
+    """Keys built to score far above everything a row saw before (by ~90-130
+    log2 units), in the first and in the second half of a later key tile: the
+    online softmax must move the row's reference and rescale O and l, with no
+    overflow and no loss of the earlier tiles' weights."""
+    if kernel == "pair" and D != 128:
+        pytest.skip("the pair kernel is built for head_dim 128")
+    L, W, Hh, H, r = 600, 2, 0, 2, 0
+    q, kc, vc = place_round(L, W, Hh, H, D, r, seed=41)
+    n1, n2, n3 = L + 5, L + 300, 17          # queries in chunk 1, 1 and 0
+    big = 8.0
+    # chunk 0, key tile 1, column 10 (first half): aligned with n1 and n3
+    kc[0, 138, 0] = (big * q[n1, 0].float()).to(torch.bfloat16)
+    kc[0, 140, 1] = (big * q[n3, 1].float()).to(torch.bfloat16)
+    # chunk 1, key tile 3, column 100 (second half): aligned with n2 and n1
+    kc[1, 484, 0] = (big * q[n2, 0].float()).to(torch.bfloat16)
+    kc[1, 490, 1] = (big * q[n1, 1].float()).to(torch.bfloat16)
+    plan = make_plan(wf, L, W, Hh, H, D, kernel)
+    o, lse = run_attn(wf, plan, r, q, kc, vc)
+    cache = oracle_cache_from_ring(kc, vc, r, W, Hh)
+    T = W * L
+    rows = np.repeat(np.arange(T), H)
+    heads = np.tile(np.arange(H), T)
+    ref, lse_ref = oracle.round_attention(cache, r, W, Hh, wi.bits(q.cpu()), rows, heads)
+    got = o.float().cpu().numpy().reshape(T * H, D)
+    assert np.isfinite(got).all()
+    targets = ((n1, 0, (0, 138)), (n2, 0, (1, 484)), (n1, 1, (1, 490)), (n3, 1, (0, 140)))
+    hit = np.zeros(T * H, bool)
+    for n, h, _ in targets:
+        hit[n * H + h] = True
+    # The big keys also pull rows that merely correlate with the targeted
+    # queries towards a single V row, so |O| reaches ~4.5 where one bf16
+    # rounding alone exceeds the 1e-2 max-abs bar: every row is held to the
+    # elementwise rounding bound, and all rows together to the mean bar.
+    v_absmax = float(vc.float().abs().max())
+    assert_attention_within_rounding(got, ref, v_absmax, "score jump D=%d" % D)
+    assert float(np.abs(got - ref).mean()) <= 1e-3
+    for n, h, key in targets:
+        v = vc[key[0], key[1], h].float().cpu().numpy()
+        assert np.max(np.abs(o[n, h].float().cpu().numpy() - v)) <= 2.0 ** -6 * np.abs(v).max()
+    lse_gpu = lse.cpu().numpy().T.reshape(-1)
+    assert np.max(np.abs(lse_gpu - lse_ref)) <= 1e-3
+    plan.destroy()
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
 def test_causality_perturbation_bit_identical(wf, kernel):
     L, W, Hh, H, D, r = 200, 4, 2, 2, 128, 6
     q, kc, vc = place_round(L, W, Hh, H, D, r, seed=5)
