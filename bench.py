@@ -19,6 +19,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -54,11 +55,26 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash():
+def strip_c_comments(text: str) -> str:
+    """C/C++ source without // and /* */ comments or blank lines (string
+    literals of the kernel sources contain no comment markers)."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
+def kernel_source_hash(read=None):
+    """Hash of the attention kernel's code (comments excluded), used to tell
+    whether the committed ncu traffic record still describes this kernel."""
     h = hashlib.sha256()
     for name in ("attn_kernel.cu", "sm100.cuh", "wf_internal.h"):
-        with open(os.path.join(ROOT, "chunk_causal_dit_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        path = os.path.join("chunk_causal_dit_b200", "csrc", name)
+        if read is None:
+            with open(os.path.join(ROOT, path)) as f:
+                text = f.read()
+        else:
+            text = read(path)
+        h.update(strip_c_comments(text).encode())
     return h.hexdigest()[:16]
 
 

@@ -61,9 +61,10 @@ static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl == kThreads * kRegsLau
               "the register re-split must add up to the launch pool");
 constexpr int kSoftmaxWarpsArrive = 8;      // sched_empty: one arrival per softmax warp
 // Pair e of a 32-pair block takes the FMA-pipe exp2 when e % kEmulatePeriod ==
-// kEmulatePeriod - 1; 0 keeps every exponential on MUFU.  Measured on B200 at
-// this design point the softmax is bound by issue and latency rather than by
-// MUFU throughput, so the default is 0 (all MUFU); 4 and 8 are tested too.
+// kEmulatePeriod - 1; 0 keeps every exponential on MUFU.  Timed on B200, sending
+// 12.5%, 25% or 33% of the exponentials to the FMA pipe made the kernel slower
+// (during its exp phase a tile's softmax is one warp per SMSP, which the extra
+// instructions lengthen more than MUFU relief shortens), so the default is 0.
 constexpr int kEmulatePeriod = 0;
 
 // F8: Q and K arrive as E4M3 codes (one byte per element, one 128-byte
