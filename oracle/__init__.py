@@ -19,6 +19,9 @@ refresh chunk is wave chunk 0 (oldest, cleanest); softmax scale ``1/sqrt(D)``;
 RMSNorm ``eps = 1e-6`` per head over D; RoPE theta 10000 with the channel
 split ``dt = D - 4*(D//6)``, ``dh = dw = 2*(D//6)``.
 
+The synthetic DiT block around the path (projections, feed-forward, norms) is
+in ``oracle/block.py``.
+
 Parity pins: ``tests/test_oracle_pins.py``.
 """
 from __future__ import annotations
@@ -82,6 +85,8 @@ def _load():
         lib.wfo_e4m3_decode.argtypes = [P, P, L]
         lib.wfo_chunk_causal_attn_rows_fp8qk.argtypes = [I, I, I, I, P, P, P, P, P, P, P, I,
                                                          I, P, P, P, P]
+        lib.wfo_qk_norm_rope_f64.argtypes = [I, I, I, P, P, P, Dd, I, I, I, Dd, P]
+        lib.wfo_qk_norm_rope_f64.restype = I
         lib.wfo_chunk_causal_attn_rows.restype = I
         lib.wfo_num_threads.restype = I
         _lib = lib

@@ -28,6 +28,11 @@
  *         channels [0,dt) rotate with t, [dt,dt+dh) with h, [dt+dh,D) with w;
  *         pair (2i, 2i+1) of an axis block of width da turns by pos*theta^(-2i/da).
  *
+ *   wfo_qk_norm_rope_f64
+ *       the same per-head RMSNorm and 3D RoPE on rows given in double (the
+ *       exact product of a projection, before any rounding); used by the
+ *       oracle of the QKV projection with the append fused into it.
+ *
  *   wfo_chunk_causal_attn_rows
  *       softmax attention of selected (query row, head) pairs over an explicit
  *       concatenation of key chunks, each tagged with its absolute chunk id.
@@ -199,6 +204,30 @@ int wfo_append(int T, int H, int D,
             for (int d = 0; d < D; ++d) v_out[base + d] = v[base + d];
         }
         free(xin); free(gam); free(nrm); free(rot);
+    }
+    return 0;
+}
+
+/* ---- norm + rope on double rows (projection output, not rounded) ------- */
+
+int wfo_qk_norm_rope_f64(int T, int H, int D, const double *x, const int32_t *pos,
+                         const float *gamma, double eps, int dt, int dh, int dw,
+                         double theta, double *y)
+{
+    if (dt + dh + dw != D || (dt | dh | dw) & 1) return -1;
+    const long rows = (long)T * H;
+#pragma omp parallel
+    {
+        double *gam = (double *)malloc(sizeof(double) * D);
+        double *nrm = (double *)malloc(sizeof(double) * D);
+#pragma omp for schedule(static)
+        for (long row = 0; row < rows; ++row) {
+            const long n = row / H, h = row % H;
+            for (int d = 0; d < D; ++d) gam[d] = (double)gamma[h * D + d];
+            wfo_rms_norm(x + row * D, gam, D, eps, nrm);
+            wfo_rope_3d(nrm, D, dt, dh, dw, theta, pos + 3 * n, y + row * D);
+        }
+        free(gam); free(nrm);
     }
     return 0;
 }
