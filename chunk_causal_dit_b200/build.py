@@ -20,7 +20,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libwf.so")
 SOURCES = ["wf_api.cu", "append_kernel.cu", "attn_kernel.cu", "attn_pair_kernel.cu",
-           "quant_fp8_kernel.cu", "noalloc.cu"]
+           "quant_fp8_kernel.cu", "noalloc.cu", "gemm_kernel.cu", "ln_kernel.cu"]
 HEADERS = ["sm100.cuh", "wf_internal.h", "exp2_poly.h"]
 
 NVCC_FLAGS = [

@@ -1,0 +1,532 @@
+// gemm_kernel.cu -- bf16 GEMM C = A B^T on tcgen05 CTA pairs, with the epilogues of the
+// DiT block fused into it.
+//
+// "Wave Forcing" (abstract) pushes every wave chunk through the layers of
+// Wan2.1-T2V-1.3B in one pass; around the chunk-causal attention those layers
+// are dense projections: the QKV projection (whose epilogue here also does the
+// per-head RMSNorm, the 3D RoPE and the ring-buffer append of the wave round,
+// so q/k/v never round-trip through HBM before the attention), the output
+// projection and the two feed-forward layers.  A is [M][K] (activations), B is
+// [N][K] (a linear layer's weight, out x in), both bf16 and K-major; the
+// accumulation is fp32 in TMEM.
+//
+// Organisation (one cluster of two CTAs per pair of SMs, persistent):
+//  * Tile = 256 rows x 256 columns per cluster; CTA rank r holds rows
+//    [128r, 128r + 128) of the tile's A and rows [128r, 128r + 128) of its B
+//    (columns of C).  The leader issues tcgen05.mma.cta_group::2 with M = 256,
+//    N = 256, K = 16; each SM reads half of the B tile, so a stage is 32 KB per
+//    SM for 512 tensor cycles of work.
+//  * A 6-stage ring of 64-deep K slices (one 128-byte swizzle row of bf16),
+//    filled by TMA; both CTAs' copies complete on the leader's barriers, the
+//    leader's commits release the stage in both CTAs.
+//  * Two 256-column fp32 accumulators in TMEM (all 512 columns): the epilogue of
+//    tile i reads one while the MMAs of tile i + 1 fill the other.
+//  * Eight epilogue warps per CTA: warp w reads TMEM lane quarter w % 4 (the
+//    lanes a warp may access) and one 128-column half of the tile; each thread
+//    owns one row of C.
+//  * Tiles are dealt statically: cluster c takes tiles c, c + clusters, ...,
+//    numbered with the column tile fastest, so the clusters working at one time
+//    share a few row blocks of A (and all of B) in L2.
+//
+// Every mbarrier wait is bounded (the plan's limit); on expiry the kernel records
+// kStatusTimeout, every role leaves its loop, the leader drains its copies and
+// MMAs, and both CTAs meet at a cluster barrier before TMEM is freed.
+#include <cuda_bf16.h>
+
+#include <atomic>
+
+#include "sm100.cuh"
+#include "wf_internal.h"
+
+namespace wf {
+
+namespace {
+
+constexpr int BM = 128;                    // rows of A per CTA (M = 256 per pair MMA)
+constexpr int BN = 256;                    // columns of C per tile (the MMA's N)
+constexpr int BK = 64;                     // K per stage: one 128-byte swizzle row of bf16
+constexpr int kStages = 6;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 32 * (2 + kEpiWarps);   // producer, MMA, 8 epilogue warps
+constexpr uint32_t kABytes = BM * BK * 2;              // 16 KB
+constexpr uint32_t kBBytes = (BN / 2) * BK * 2;        // 16 KB: this CTA's 128 rows of B
+constexpr uint32_t kStageBytes = kABytes + kBBytes;
+constexpr uint32_t kTabOff = kStages * kStageBytes;    // RoPE (cos, sin) tables, QKV only
+constexpr int kTabMax = 3072;                          // float2 entries (24 KB)
+constexpr uint32_t kTmemCols = 512;
+constexpr unsigned long long kDrainLimit = 1ull << 32;
+
+template <int Epi>
+__host__ __device__ constexpr uint32_t bar_off()
+{
+    return Epi == kEpiQkvAppend ? kTabOff + kTabMax * 8 : kTabOff;
+}
+template <int Epi>
+__host__ __device__ constexpr uint32_t smem_bytes()
+{
+    return bar_off<Epi>() + 256 + 1024;
+}
+static_assert(smem_bytes<kEpiQkvAppend>() <= 232448, "shared memory per CTA");
+
+struct Bars {
+    static constexpr int full = 0, empty = kStages, acc_full = 2 * kStages,
+                         acc_empty = 2 * kStages + 2, drain = 2 * kStages + 4,
+                         count = 2 * kStages + 5;
+};
+static_assert(Bars::count * 8 + 8 <= 256, "barrier block");
+
+enum : uint32_t {
+    kWhereProducer = 21, kWhereMmaFull = 22, kWhereMmaAcc = 23, kWhereEpi = 24, kWhereDrain = 25,
+};
+
+struct Ctl {
+    volatile uint32_t *abort;
+    uint32_t peer_abort;      // the other CTA's abort word (shared::cluster address)
+    DeviceWords *words;
+    unsigned long long limit;
+};
+
+// Bounded wait with cluster-scope acquire (phases may be completed from the peer CTA).
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ctl &ctl,
+                                         uint32_t where, bool drain = false)
+{
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const long long t0 = clock64();
+    const unsigned long long limit = drain ? kDrainLimit : ctl.limit;
+    while (true) {
+#pragma unroll 1
+        for (int k = 0; k < 32; ++k)
+            if (mbar_try_wait_cluster(bar, parity)) return true;
+        if (!drain && *ctl.abort) return false;
+        if (static_cast<unsigned long long>(clock64() - t0) > limit) {
+            *ctl.abort = 1u;
+            st_cluster_u32(ctl.peer_abort, 1u);     // the pair stops together
+            atomicOr(&ctl.words->status, kStatusTimeout);
+            atomicCAS(&ctl.words->timeout_where, 0u, where);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ float gelu_tanh(float x)
+{
+    // 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))), the tanh form of GELU
+    const float u = 0.7978845608028654f * fmaf(0.044715f * x, x * x, x);
+    return 0.5f * x * (1.0f + tanhf(u));
+}
+
+__device__ __forceinline__ uint4 pack8(const float *y)
+{
+    uint4 u;
+    u.x = pack_bf16x2(y[0], y[1]);
+    u.y = pack_bf16x2(y[2], y[3]);
+    u.z = pack_bf16x2(y[4], y[5]);
+    u.w = pack_bf16x2(y[6], y[7]);
+    return u;
+}
+
+__device__ __forceinline__ void unpack8(const uint4 &u, float *x)
+{
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        x[2 * i] = __uint_as_float(w[i] << 16);
+        x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
+// 32 columns [c, c + 32) of one row: bias, activation / gated residual, bf16 store.
+template <int Epi>
+__device__ __forceinline__ void finish32(const GemmParams &p, const uint32_t (&r)[32], long row,
+                                         int c, const float *gate_row)
+{
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+    if (p.bias != nullptr) {
+        const float4 *b4 = reinterpret_cast<const float4 *>(p.bias + c);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float4 b = __ldg(b4 + j);
+            v[4 * j] += b.x;
+            v[4 * j + 1] += b.y;
+            v[4 * j + 2] += b.z;
+            v[4 * j + 3] += b.w;
+        }
+    }
+    if constexpr (Epi == kEpiGeluTanh) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = gelu_tanh(v[i]);
+    }
+    if constexpr (Epi == kEpiGatedResidual) {
+        const uint4 *r4 = reinterpret_cast<const uint4 *>(p.resid + row * p.N + c);
+        const float4 *g4 = reinterpret_cast<const float4 *>(gate_row + c);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float x[8];
+            unpack8(__ldg(r4 + j), x);
+            const float4 ga = __ldg(g4 + 2 * j), gb = __ldg(g4 + 2 * j + 1);
+            const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[8 * j + e] = fmaf(g[e], v[8 * j + e], x[e]);
+        }
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(p.c + row * p.N + c);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) dst[j] = pack8(v + 8 * j);
+}
+
+// Linear epilogues: this thread's row, 128 columns from col0 (TMEM at taddr).
+template <int Epi>
+__device__ __forceinline__ void epi_linear(const GemmParams &p, uint32_t taddr, long row, int col0)
+{
+    const bool row_ok = row < p.M;
+    const float *gate_row = nullptr;
+    if constexpr (Epi == kEpiGatedResidual)
+        gate_row = p.gate + (row_ok ? row / p.rows_per_group : 0) * static_cast<long>(p.N);
+#pragma unroll 1
+    for (int h = 0; h < 2; ++h) {
+        uint32_t r0[32], r1[32];
+        tmem_ld32(taddr + 64 * h, r0);
+        tmem_ld32(taddr + 64 * h + 32, r1);
+        tmem_wait_ld();
+        const int c = col0 + 64 * h;
+        if (!row_ok) continue;
+        if (c < p.N) finish32<Epi>(p, r0, row, c, gate_row);
+        if (c + 32 < p.N) finish32<Epi>(p, r1, row, c + 32, gate_row);
+    }
+}
+
+// QKV epilogue: this thread's wave token `row`, 128 columns from col0, i.e. 128 / D
+// heads of one of q, k, v (the column split puts q, k and v at multiples of H*D,
+// which the host keeps a multiple of 128).  q and k: RMSNorm over the head with
+// gain gamma, then the 3D RoPE with the (cos, sin) tables, one rounding to bf16;
+// q goes to q_out [T][H][D], k and v to row ic of the ring slot of the token's
+// chunk, (round + c) mod R, as the stand-alone append kernel writes them.
+template <int D>
+__device__ __forceinline__ void epi_qkv(const GemmParams &p, uint32_t taddr, long row, int col0,
+                                        const float2 *tab)
+{
+    constexpr int kHeads = 128 / D;
+    const int HD = p.H * D;
+    const bool ok = row < p.M && col0 < p.N;
+    const int which = col0 / HD;                 // 0 q, 1 k, 2 v
+    const int h0 = (col0 - which * HD) / D;
+    const long n = ok ? row : 0;                 // rows past M store nothing
+    const int c = static_cast<int>(n / p.L);
+    const int ic = static_cast<int>(n - static_cast<long>(c) * p.L);
+    const int hw = p.rope.gh * p.rope.gw;
+    const int f = ic / hw;
+    const int rem = ic - f * hw;
+    const int y = rem / p.rope.gw;
+    const int x = rem - y * p.rope.gw;
+    const int nt = p.rope.dt / 2, nh = p.rope.dh / 2, nw = p.rope.dw / 2;
+    const int nfr = p.W * p.rope.F;
+    // table index of pair pr: it + pr (t block), ih + pr (h block), iw + pr (w block)
+    const int it = (c * p.rope.F + f) * nt;
+    const int ih = nfr * nt + y * nh - nt;
+    const int iw = nfr * nt + p.rope.gh * nh + x * nw - nt - nh;
+    const int slot = ring_slot(p.round + c, p.R);
+#pragma unroll 1
+    for (int hh = 0; hh < kHeads; ++hh) {
+        uint32_t r[D / 32][32];
+#pragma unroll
+        for (int j = 0; j < D / 32; ++j) tmem_ld32(taddr + hh * D + 32 * j, r[j]);
+        tmem_wait_ld();
+        if (!ok) continue;
+        const int h = h0 + hh;
+        const int col = col0 + hh * D;
+        float v[D];
+#pragma unroll
+        for (int i = 0; i < D; ++i) v[i] = __uint_as_float(r[i / 32][i % 32]);
+        if (p.bias != nullptr) {
+            const float4 *b4 = reinterpret_cast<const float4 *>(p.bias + col);
+#pragma unroll
+            for (int j = 0; j < D / 4; ++j) {
+                const float4 b = __ldg(b4 + j);
+                v[4 * j] += b.x;
+                v[4 * j + 1] += b.y;
+                v[4 * j + 2] += b.z;
+                v[4 * j + 3] += b.w;
+            }
+        }
+        uint16_t *dst;
+        if (which == 0)
+            dst = p.q_out + (n * p.H + h) * D;
+        else
+            dst = (which == 1 ? p.k_cache : p.v_cache) +
+                  ((static_cast<long>(slot) * p.L + ic) * p.H + h) * D;
+        if (which < 2) {
+            float ss = 0.0f;
+#pragma unroll
+            for (int i = 0; i < D; ++i) ss = fmaf(v[i], v[i], ss);
+            const float rs = rsqrtf(ss * (1.0f / D) + p.eps);
+            const float4 *g4 =
+                reinterpret_cast<const float4 *>((which ? p.gamma_k : p.gamma_q) + h * D);
+#pragma unroll
+            for (int j = 0; j < D / 4; ++j) {
+                const float4 g = __ldg(g4 + j);
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int pr = 2 * j + e;
+                    const float a = v[2 * pr] * rs * (e ? g.z : g.x);
+                    const float b = v[2 * pr + 1] * rs * (e ? g.w : g.y);
+                    const float2 cs = tab[pr < nt ? it + pr : (pr < nt + nh ? ih + pr : iw + pr)];
+                    v[2 * pr] = a * cs.x - b * cs.y;
+                    v[2 * pr + 1] = a * cs.y + b * cs.x;
+                }
+            }
+        }
+        uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+        for (int j = 0; j < D / 8; ++j) d4[j] = pack8(v + 8 * j);
+    }
+}
+
+template <int Epi, int D>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                 const GemmParams p)
+{
+    using B = Bars;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = smem_addr(smem);
+    const uint32_t sbar = sbase + bar_off<Epi>();
+    auto bar = [&](int i) -> uint32_t { return sbar + 8u * static_cast<uint32_t>(i); };
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + bar_off<Epi>() + 8 * B::count);
+    volatile uint32_t *abort_flag = tmem_slot + 1;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+    const int cid = static_cast<int>(cluster_id_x());
+    const int ncl = static_cast<int>(nclusters_x());
+    auto lead = [&](int i) -> uint32_t { return map_to_rank(bar(i), 0); };
+    const int nk = (p.K + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(bar(B::full + s), 1);
+            mbar_init(bar(B::empty + s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar(B::acc_full + b), 1);
+            mbar_init(bar(B::acc_empty + b), 2 * kEpiWarps);   // both CTAs' epilogue warps
+        }
+        mbar_init(bar(B::drain), 1);
+        *abort_flag = 0u;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(smem_addr(tmem_slot), kTmemCols);
+        tmem_relinquish_pair();
+    }
+    if constexpr (Epi == kEpiQkvAppend) {
+        // (cos, sin) of every (frame, t pair), (row y, h pair), (column x, w pair): the
+        // angle pos * omega in fp64, reduced to [-pi, pi] in fp64, then fp32 sincos
+        if (warp >= 2) {
+            float2 *tab = reinterpret_cast<float2 *>(smem + kTabOff);
+            const int nt = p.rope.dt / 2, nh = p.rope.dh / 2, nw = p.rope.dw / 2;
+            const int n_t = p.W * p.rope.F * nt, n_h = p.rope.gh * nh;
+            for (int i = threadIdx.x - 64; i < p.n_tab; i += 32 * kEpiWarps) {
+                int pr;
+                long pos;
+                if (i < n_t) {
+                    const int fi = i / nt;
+                    pr = i - fi * nt;
+                    pos = p.round * p.rope.F + fi;
+                } else if (i < n_t + n_h) {
+                    const int j = i - n_t, yy = j / nh;
+                    pr = nt + (j - yy * nh);
+                    pos = yy;
+                } else {
+                    const int j = i - n_t - n_h, xx = j / nw;
+                    pr = nt + nh + (j - xx * nw);
+                    pos = xx;
+                }
+                const double ang = static_cast<double>(pos) * p.rope.omega[pr];
+                const double k = rint(ang * 0.15915494309189535);   // 1 / (2 pi)
+                const float red = static_cast<float>(fma(-k, 6.283185307179586, ang));
+                float sn, cs;
+                sincosf(red, &sn, &cs);
+                tab[i] = make_float2(cs, sn);
+            }
+        }
+    }
+    tc_fence_before();
+    cluster_sync();                 // barriers, TMEM address and tables ready in both CTAs
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const Ctl ctl{abort_flag, map_to_rank(smem_addr(const_cast<uint32_t *>(abort_flag)), rank ^ 1u),
+                  p.words, p.wait_limit};
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer (both CTAs) ----------------
+            tma_prefetch_desc(&tmap_a);
+            tma_prefetch_desc(&tmap_b);
+            uint32_t it = 0;
+            bool ok = true;
+            for (int t = cid; ok && t < p.n_tiles; t += ncl) {
+                const int mb = t / p.n_ntiles, nb = t - mb * p.n_ntiles;
+                const int arow = mb * 2 * BM + static_cast<int>(rank) * BM;
+                const int brow = nb * BN + static_cast<int>(rank) * (BN / 2);
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const uint32_t st = it % kStages;
+                    if (!(ok = wait_bar(bar(B::empty + st), ((it / kStages) & 1u) ^ 1u, ctl,
+                                        kWhereProducer)))
+                        break;
+                    if (leader) mbar_arrive_expect_tx(bar(B::full + st), 2 * kStageBytes);
+                    const uint32_t dst = sbase + st * kStageBytes;
+                    tma_load_2d_pair(dst, &tmap_a, lead(B::full + st), kb * BK, arow);
+                    tma_load_2d_pair(dst + kABytes, &tmap_b, lead(B::full + st), kb * BK, brow);
+                }
+            }
+            if (!ok && leader) {
+                // both CTAs' copies complete on the leader's barriers: let them land
+                for (uint32_t s = 0; s < static_cast<uint32_t>(kStages); ++s) {
+                    const uint32_t fills = (it + kStages - 1 - s) / kStages;
+                    if (fills)
+                        wait_bar(bar(B::full + s), (fills - 1) & 1u, ctl, kWhereDrain, true);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            // ---------------- MMA issuer (leader CTA, for the pair) ----------------
+            constexpr uint32_t idesc = idesc_bf16_f32(2 * BM, BN, false);
+            constexpr uint32_t hi = sw128_desc_hi(1024);
+            uint32_t it = 0, acc_it = 0;
+            bool ok = true;
+            for (int t = cid; ok && t < p.n_tiles; t += ncl, ++acc_it) {
+                const uint32_t b = acc_it & 1u;
+                if (!(ok = wait_bar(bar(B::acc_empty + b), ((acc_it >> 1) & 1u) ^ 1u, ctl,
+                                    kWhereMmaAcc)))
+                    break;
+                tc_fence_after();
+                const uint32_t d = tmem + b * BN;
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const uint32_t st = it % kStages;
+                    if (!(ok = wait_bar(bar(B::full + st), (it / kStages) & 1u, ctl, kWhereMmaFull)))
+                        break;
+                    tc_fence_after();
+                    const uint32_t alo = sw128_desc_lo(sbase + st * kStageBytes, 16);
+                    const uint32_t blo = sw128_desc_lo(sbase + st * kStageBytes + kABytes, 16);
+#pragma unroll
+                    for (int s = 0; s < BK / 16; ++s)
+                        umma_ss_pair(d, desc_join(alo + ((s * 32) >> 4), hi),
+                                     desc_join(blo + ((s * 32) >> 4), hi), idesc,
+                                     (kb | s) ? 1u : 0u);
+                    umma_commit_pair_mc(bar(B::empty + st), 0x3);
+                }
+                if (!ok) break;
+                umma_commit_pair_mc(bar(B::acc_full + b), 0x3);
+            }
+            // every MMA of the pair completes before either CTA releases TMEM
+            umma_commit_pair_mc(bar(B::drain), 0x1);
+            wait_bar(bar(B::drain), 0u, ctl, kWhereDrain, true);
+        }
+    } else {
+        // ---------------- epilogue: 8 warps, one row of C per thread ----------------
+        const int lq = warp & 3;                   // TMEM lane quarter of this warp
+        const int half = (warp - 2) >> 2;          // 128-column half of the tile
+        const float2 *tab = reinterpret_cast<const float2 *>(smem + kTabOff);
+        uint32_t acc_it = 0;
+        for (int t = cid; t < p.n_tiles; t += ncl, ++acc_it) {
+            const uint32_t b = acc_it & 1u;
+            bool ok = wait_bar(bar(B::acc_full + b), (acc_it >> 1) & 1u, ctl, kWhereEpi);
+            ok = __all_sync(0xFFFFFFFFu, ok);
+            if (!ok) break;
+            tc_fence_after();
+            const int mb = t / p.n_ntiles, nb = t - mb * p.n_ntiles;
+            const long row = static_cast<long>(mb) * 2 * BM + rank * BM + lq * 32 + lane;
+            const int col0 = nb * BN + half * (BN / 2);
+            const uint32_t taddr =
+                tmem + (static_cast<uint32_t>(lq * 32) << 16) + b * BN + half * (BN / 2);
+            if constexpr (Epi == kEpiQkvAppend)
+                epi_qkv<D>(p, taddr, row, col0, tab);
+            else
+                epi_linear<Epi>(p, taddr, row, col0);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(lead(B::acc_empty + b));
+        }
+    }
+
+    // both CTAs stop sending to each other before either frees TMEM or exits
+    tc_fence_before();
+    __syncwarp();
+    cluster_sync();
+    tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        tmem_dealloc_pair(tmem, kTmemCols);
+    }
+}
+
+template <int Epi, int D>
+cudaError_t launch_gemm_t(const CUtensorMap &ma, const CUtensorMap &mb, const GemmParams &p,
+                          cudaStream_t stream)
+{
+    constexpr int kMaxDevices = 64;
+    static std::atomic<int> resident_pairs[kMaxDevices];
+    auto kern = gemm_pair_kernel<Epi, D>;
+    constexpr uint32_t smem = smem_bytes<Epi>();
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(2, 1, 1);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return cudaErrorInvalidDevice;
+    // clusters of two that can be resident at once (one CTA per SM), once per device
+    int resident = resident_pairs[dev].load(std::memory_order_relaxed);
+    if (resident < 1) {
+        if (cudaOccupancyMaxActiveClusters(&resident, kern, &cfg) != cudaSuccess || resident < 1) {
+            (void)cudaGetLastError();
+            return cudaErrorInvalidConfiguration;
+        }
+        resident_pairs[dev].store(resident, std::memory_order_relaxed);
+    }
+    const int n_clusters = p.n_tiles < resident ? p.n_tiles : resident;
+    cfg.gridDim = dim3(2 * n_clusters, 1, 1);
+    e = cudaLaunchKernelEx(&cfg, kern, ma, mb, p);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// Tensor maps: ma over A [M][K], mb over B [N][K], both bf16 with a 64 x 128 box and
+// the 128-byte swizzle.
+cudaError_t launch_gemm(const CUtensorMap &ma, const CUtensorMap &mb, const GemmParams &p, int epi,
+                        cudaStream_t stream)
+{
+    if (p.n_tiles == 0) return cudaSuccess;
+    switch (epi) {
+    case kEpiStore: return launch_gemm_t<kEpiStore, 128>(ma, mb, p, stream);
+    case kEpiGeluTanh: return launch_gemm_t<kEpiGeluTanh, 128>(ma, mb, p, stream);
+    case kEpiGatedResidual: return launch_gemm_t<kEpiGatedResidual, 128>(ma, mb, p, stream);
+    case kEpiQkvAppend:
+        return p.D == 128 ? launch_gemm_t<kEpiQkvAppend, 128>(ma, mb, p, stream)
+                          : launch_gemm_t<kEpiQkvAppend, 64>(ma, mb, p, stream);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+int gemm_tab_max() { return kTabMax; }
+
+}  // namespace wf

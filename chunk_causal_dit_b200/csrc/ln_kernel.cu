@@ -1,0 +1,107 @@
+// ln_kernel.cu -- LayerNorm (no affine) with per-chunk adaLN modulation, the step
+// before the QKV projection and before the feed-forward layer of a DiT block.
+//
+// The wave of "Wave Forcing" (abstract) holds chunks at different denoising
+// steps, so each chunk carries its own modulation: row n of the wave uses row
+// n / rows_per_group of shift and scale.  y = (x - mean) / sqrt(var + eps) *
+// (1 + scale) + shift, with the mean and the (biased) variance over the row,
+// fp32 arithmetic and one rounding to bf16.
+//
+// HBM-bound: 2 bytes read and 2 written per element (the modulation tables are
+// small and stay in L1/L2).  One warp per row; lane l owns the 16-byte pieces
+// l, l + 32, ... of the row, all loaded before the reductions.
+#include <cuda_bf16.h>
+
+#include "sm100.cuh"
+#include "wf_internal.h"
+
+namespace wf {
+
+namespace {
+
+constexpr int kMaxPieces = 24;      // 16-byte pieces per lane: C <= 32 * 24 * 8 = 6144
+constexpr int kRowsPerBlock = 8;
+
+__global__ void __launch_bounds__(32 * kRowsPerBlock)
+layer_norm_modulate_kernel(const uint16_t *__restrict__ x, const float *__restrict__ shift,
+                           const float *__restrict__ scale, uint16_t *__restrict__ y, long M, int C,
+                           int rows_per_group, float eps)
+{
+    const int lane = threadIdx.x & 31;
+    const long row = static_cast<long>(blockIdx.x) * kRowsPerBlock + (threadIdx.x >> 5);
+    if (row >= M) return;                   // whole warps leave together
+    const int pieces = C / 8;
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + row * C);
+    uint4 w[kMaxPieces];
+#pragma unroll
+    for (int i = 0; i < kMaxPieces; ++i) {
+        const int j = lane + 32 * i;
+        w[i] = j < pieces ? __ldcs(src + j) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    float s = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kMaxPieces; ++i) {
+        const uint32_t u[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            s += __uint_as_float(u[e] << 16) + __uint_as_float(u[e] & 0xFFFF0000u);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+    const float mean = s / static_cast<float>(C);
+    float v = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kMaxPieces; ++i) {
+        if (lane + 32 * i >= pieces) break;
+        const uint32_t u[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float a = __uint_as_float(u[e] << 16) - mean;
+            const float b = __uint_as_float(u[e] & 0xFFFF0000u) - mean;
+            v = fmaf(a, a, fmaf(b, b, v));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    const float rstd = rsqrtf(v / static_cast<float>(C) + eps);
+    const long g = row / rows_per_group;
+    const float4 *sh4 = reinterpret_cast<const float4 *>(shift + g * C);
+    const float4 *sc4 = reinterpret_cast<const float4 *>(scale + g * C);
+    uint4 *dst = reinterpret_cast<uint4 *>(y + row * C);
+#pragma unroll
+    for (int i = 0; i < kMaxPieces; ++i) {
+        const int j = lane + 32 * i;
+        if (j >= pieces) break;
+        const uint32_t u[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+        const float4 sa = __ldg(sh4 + 2 * j), sb = __ldg(sh4 + 2 * j + 1);
+        const float4 ca = __ldg(sc4 + 2 * j), cb = __ldg(sc4 + 2 * j + 1);
+        const float shv[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
+        const float scv[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float a = (__uint_as_float(u[e] << 16) - mean) * rstd;
+            const float b = (__uint_as_float(u[e] & 0xFFFF0000u) - mean) * rstd;
+            o[e] = pack_bf16x2(fmaf(a, 1.0f + scv[2 * e], shv[2 * e]),
+                               fmaf(b, 1.0f + scv[2 * e + 1], shv[2 * e + 1]));
+        }
+        dst[j] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+}  // namespace
+
+int ln_max_channels() { return 32 * kMaxPieces * 8; }
+
+cudaError_t launch_layer_norm_modulate(const uint16_t *x, const float *shift, const float *scale,
+                                       uint16_t *y, long M, int C, int rows_per_group, float eps,
+                                       cudaStream_t stream)
+{
+    if (M == 0) return cudaSuccess;
+    const dim3 grid(static_cast<unsigned>((M + kRowsPerBlock - 1) / kRowsPerBlock));
+    layer_norm_modulate_kernel<<<grid, 32 * kRowsPerBlock, 0, stream>>>(x, shift, scale, y, M, C,
+                                                                        rows_per_group, eps);
+    return cudaGetLastError();
+}
+
+}  // namespace wf

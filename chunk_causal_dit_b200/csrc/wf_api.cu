@@ -23,6 +23,13 @@ cudaError_t launch_quantize_rows(const uint16_t *q, uint8_t *q8, float *scale, l
                                  int D, cudaStream_t stream);
 cudaError_t launch_quantize_tiles(const uint16_t *k, uint8_t *k8, float *scale, long first_chunk,
                                   int n_chunks, int L, int H, int R, int D, cudaStream_t stream);
+cudaError_t launch_gemm(const CUtensorMap &ma, const CUtensorMap &mb, const GemmParams &p, int epi,
+                        cudaStream_t stream);
+int gemm_tab_max();
+cudaError_t launch_layer_norm_modulate(const uint16_t *x, const float *shift, const float *scale,
+                                       uint16_t *y, long M, int C, int rows_per_group, float eps,
+                                       cudaStream_t stream);
+int ln_max_channels();
 }  // namespace wf
 
 namespace {
@@ -101,6 +108,33 @@ bool encode_map_u8(CUtensorMap *map, const void *base, int D, int H, int n2, int
 }
 
 bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// 2-D map over a row-major [rows][cols] bf16 matrix (a GEMM operand, K = cols
+// innermost): box = 64 columns x 128 rows, 128-byte swizzle, out-of-range reads 0.
+bool encode_map_2d(CUtensorMap *map, const void *base, long rows, long cols)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+    const cuuint32_t box[2] = {64, 128};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// Tile counts of a GEMM (256 x 256 tiles); false if they do not fit an int.
+bool gemm_tiles(long M, long N, wf::GemmParams &g)
+{
+    const long nt = (N + 255) / 256, mt = (M + 255) / 256;
+    if (mt * nt >= INT_MAX) return false;
+    g.n_ntiles = static_cast<int>(nt);
+    g.n_tiles = static_cast<int>(mt * nt);
+    return true;
+}
 
 int check_device(const wf_plan_s *p)
 {
@@ -414,6 +448,104 @@ int wf_chunk_causal_attn_fp8qk(wf_plan_t p, long round, const void *q8, const fl
     a.k_scale = k_scale;
     const int grid = a.n_units < p->num_sms ? a.n_units : p->num_sms;
     cudaError_t e = wf::launch_attn_fp8qk(mq, mk, mv, a, grid, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? WF_OK : WF_ERR_CUDA;
+}
+
+int wf_linear(wf_plan_t p, int M, int N, int K, const void *x, const void *w, const float *bias,
+              int epilogue, const float *gate, const void *resid, int rows_per_group, void *y,
+              void *stream)
+{
+    if (p == nullptr || M < 0 || N < 32 || K < 8 || N % 32 || K % 8) return WF_ERR_INVALID_ARG;
+    if (epilogue < WF_EPI_STORE || epilogue > WF_EPI_GATED_RESIDUAL) return WF_ERR_INVALID_ARG;
+    if (M == 0) return WF_OK;                        // nothing to compute, nothing is read
+    if (!x || !w || !y || !aligned16(x) || !aligned16(w) || !aligned16(y) || !aligned16(bias))
+        return WF_ERR_INVALID_ARG;
+    if (epilogue == WF_EPI_GATED_RESIDUAL &&
+        (!gate || !resid || !aligned16(gate) || !aligned16(resid) || rows_per_group < 1))
+        return WF_ERR_INVALID_ARG;
+    if (int s = check_device(p)) return s;
+
+    wf::GemmParams g{};
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    if (!gemm_tiles(M, N, g)) return WF_ERR_INVALID_ARG;
+    g.bias = bias;
+    g.c = static_cast<uint16_t *>(y);
+    g.resid = static_cast<const uint16_t *>(resid);
+    g.gate = gate;
+    g.rows_per_group = rows_per_group < 1 ? 1 : rows_per_group;
+    g.wait_limit = p->wait_limit;
+    g.words = p->words;
+    CUtensorMap ma, mb;
+    if (!encode_map_2d(&ma, x, M, K) || !encode_map_2d(&mb, w, N, K)) return WF_ERR_CUDA;
+    cudaError_t e = wf::launch_gemm(ma, mb, g, epilogue, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? WF_OK : WF_ERR_CUDA;
+}
+
+int wf_qkv_proj_norm_rope_append(wf_plan_t p, long round, int hidden, const void *x,
+                                 const void *w_qkv, const float *b_qkv, const float *gamma_q,
+                                 const float *gamma_k, void *q_out, void *k_cache, void *v_cache,
+                                 void *stream)
+{
+    if (p == nullptr || round < 0 || hidden < 8 || hidden % 8) return WF_ERR_INVALID_ARG;
+    if (!x || !w_qkv || !gamma_q || !gamma_k || !q_out || !k_cache || !v_cache)
+        return WF_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_qkv) || !aligned16(b_qkv) || !aligned16(gamma_q) ||
+        !aligned16(gamma_k) || !aligned16(q_out) || !aligned16(k_cache) || !aligned16(v_cache))
+        return WF_ERR_INVALID_ARG;
+    if (p->rope.F == 0) return WF_ERR_INVALID_ARG;            // positions come from the grid
+    if ((round + p->W) > static_cast<long>(INT_MAX / p->rope.F)) return WF_ERR_INVALID_ARG;
+    if ((p->H * p->D) % 128) return WF_ERR_UNSUPPORTED;      // q | k | v split on 128 columns
+    const long n_tab = static_cast<long>(p->W) * p->rope.F * (p->rope.dt / 2) +
+                       static_cast<long>(p->rope.gh) * (p->rope.dh / 2) +
+                       static_cast<long>(p->rope.gw) * (p->rope.dw / 2);
+    if (n_tab > wf::gemm_tab_max()) return WF_ERR_UNSUPPORTED;
+    if (int s = check_device(p)) return s;
+
+    const long T = static_cast<long>(p->L) * p->W;
+    wf::GemmParams g{};
+    g.M = static_cast<int>(T);
+    g.N = 3 * p->H * p->D;
+    g.K = hidden;
+    if (!gemm_tiles(g.M, g.N, g)) return WF_ERR_INVALID_ARG;
+    g.bias = b_qkv;
+    g.q_out = static_cast<uint16_t *>(q_out);
+    g.k_cache = static_cast<uint16_t *>(k_cache);
+    g.v_cache = static_cast<uint16_t *>(v_cache);
+    g.gamma_q = gamma_q;
+    g.gamma_k = gamma_k;
+    g.round = round;
+    g.L = p->L;
+    g.W = p->W;
+    g.R = p->R;
+    g.H = p->H;
+    g.D = p->D;
+    g.eps = static_cast<float>(p->eps);
+    g.rope = p->rope;
+    g.n_tab = static_cast<int>(n_tab);
+    g.wait_limit = p->wait_limit;
+    g.words = p->words;
+    CUtensorMap ma, mb;
+    if (!encode_map_2d(&ma, x, T, hidden) || !encode_map_2d(&mb, w_qkv, g.N, hidden))
+        return WF_ERR_CUDA;
+    cudaError_t e =
+        wf::launch_gemm(ma, mb, g, wf::kEpiQkvAppend, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? WF_OK : WF_ERR_CUDA;
+}
+
+int wf_layer_norm_modulate(wf_plan_t p, int M, int C, const void *x, const float *shift,
+                           const float *scale, int rows_per_group, void *y, void *stream)
+{
+    if (p == nullptr || M < 0 || C < 8 || C % 8 || rows_per_group < 1) return WF_ERR_INVALID_ARG;
+    if (C > wf::ln_max_channels()) return WF_ERR_UNSUPPORTED;
+    if (!x || !shift || !scale || !y || !aligned16(x) || !aligned16(shift) || !aligned16(scale) ||
+        !aligned16(y))
+        return WF_ERR_INVALID_ARG;
+    if (int s = check_device(p)) return s;
+    cudaError_t e = wf::launch_layer_norm_modulate(
+        static_cast<const uint16_t *>(x), shift, scale, static_cast<uint16_t *>(y), M, C,
+        rows_per_group, 1e-6f, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? WF_OK : WF_ERR_CUDA;
 }
 

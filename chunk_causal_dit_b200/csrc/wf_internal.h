@@ -85,6 +85,34 @@ struct AttnParams {
     const float *k_scale;     // FP8 Q.K^T only: [R][n_ktiles][H] per-tile K scales
 };
 
+// Epilogues of the bf16 GEMM (the first three are WF_EPI_* of the C ABI).
+enum GemmEpilogue : int {
+    kEpiStore = 0,            // C = A B^T + bias
+    kEpiGeluTanh = 1,         // C = gelu_tanh(A B^T + bias)
+    kEpiGatedResidual = 2,    // C = resid + gate[row / rows_per_group] * (A B^T + bias)
+    kEpiQkvAppend = 3,        // QKV projection: RMSNorm + RoPE on q/k, q -> q_out, k/v -> ring
+};
+
+struct GemmParams {
+    int M, N, K;
+    int n_ntiles, n_tiles;    // 256-column tiles per row block; all tiles (256 x 256)
+    const float *bias;        // [N] or nullptr
+    uint16_t *c;              // [M][N] bf16 (linear epilogues)
+    const uint16_t *resid;    // [M][N] bf16 (gated residual)
+    const float *gate;        // [G][N] (gated residual)
+    int rows_per_group;
+    // QKV epilogue: columns [0,HD) q, [HD,2HD) k, [2HD,3HD) v; rows are wave tokens
+    uint16_t *q_out, *k_cache, *v_cache;
+    const float *gamma_q, *gamma_k;
+    long round;
+    int L, W, R, H, D;
+    float eps;
+    RopeParams rope;
+    int n_tab;                // (cos, sin) table entries: W*F*dt/2 + gh*dh/2 + gw*dw/2
+    unsigned long long wait_limit;
+    DeviceWords *words;
+};
+
 }  // namespace wf
 
 struct wf_plan_s {

@@ -20,6 +20,7 @@ import numpy as np
 import torch
 
 STREAM_Q, STREAM_K, STREAM_V, STREAM_CACHE, STREAM_GAMMA = 0, 1, 2, 3, 4
+STREAM_X, STREAM_W, STREAM_BIAS, STREAM_MOD = 5, 6, 7, 8
 
 
 @dataclass(frozen=True)
@@ -116,6 +117,56 @@ def history_prefill(w: Workload, n_chunks: Optional[int] = None, seed: int = 0,
     g = torch.randn((2, n, w.L, w.H, w.D), generator=_gen(seed + 1009 * salt, STREAM_CACHE),
                     dtype=torch.float32).to(torch.bfloat16)
     return g[0].contiguous(), g[1].contiguous()
+
+
+def bf16_weight(out_features: int, in_features: int, seed: int, salt: int = 0) -> torch.Tensor:
+    """A random-init linear weight [out, in]: N(0, 1/in) draws rounded to bf16."""
+    g = _gen(seed + 1009 * salt, STREAM_W)
+    w = torch.randn((out_features, in_features), generator=g, dtype=torch.float32)
+    return (w * in_features ** -0.5).to(torch.bfloat16)
+
+
+def f32_vector(shape, scale: float, seed: int, stream: int, salt: int = 0) -> torch.Tensor:
+    """float32 N(0, scale^2) draws (biases, modulation tables)."""
+    g = _gen(seed + 1009 * salt, stream)
+    return torch.randn(tuple(shape), generator=g, dtype=torch.float32) * scale
+
+
+# Hidden and feed-forward widths of the Wan2.1-T2V-1.3B block (12 heads x 128 = 1536).
+WAN13B_HIDDEN = 1536
+WAN13B_FFN = 8960
+
+
+@dataclass
+class BlockInputs:
+    x: torch.Tensor          # bf16 [T, C] residual stream entering the block
+    w_qkv: torch.Tensor      # bf16 [3HD, C]
+    b_qkv: torch.Tensor      # f32 [3HD]
+    w_o: torch.Tensor        # bf16 [C, HD]
+    b_o: torch.Tensor        # f32 [C]
+    w_1: torch.Tensor        # bf16 [F, C]
+    b_1: torch.Tensor        # f32 [F]
+    w_2: torch.Tensor        # bf16 [C, F]
+    b_2: torch.Tensor        # f32 [C]
+    mod: torch.Tensor        # f32 [6, n_wave, C]: shift/scale/gate of attention, then of the FFN
+    gamma_q: torch.Tensor    # f32 [H, D]
+    gamma_k: torch.Tensor    # f32 [H, D]
+
+
+def block_inputs(w: Workload, hidden: int, ffn: int, seed: int = 0) -> BlockInputs:
+    """Random-init weights and one wave's residual stream for a DiT block of width
+    ``hidden`` (= H*D for the Wan shapes) and feed-forward width ``ffn``.  Each wave
+    chunk gets its own modulation rows (its own denoising step)."""
+    HD = w.H * w.D
+    gq, gk = gains(w.H, w.D, seed)
+    return BlockInputs(
+        x=bf16_normal((w.T, hidden), seed, STREAM_X),
+        w_qkv=bf16_weight(3 * HD, hidden, seed, 1), b_qkv=f32_vector((3 * HD,), 0.02, seed, STREAM_BIAS, 1),
+        w_o=bf16_weight(hidden, HD, seed, 2), b_o=f32_vector((hidden,), 0.02, seed, STREAM_BIAS, 2),
+        w_1=bf16_weight(ffn, hidden, seed, 3), b_1=f32_vector((ffn,), 0.02, seed, STREAM_BIAS, 3),
+        w_2=bf16_weight(hidden, ffn, seed, 4), b_2=f32_vector((hidden,), 0.02, seed, STREAM_BIAS, 4),
+        mod=f32_vector((6, w.n_wave, hidden), 0.1, seed, STREAM_MOD),
+        gamma_q=gq, gamma_k=gk)
 
 
 def bits(t: torch.Tensor) -> np.ndarray:

@@ -26,6 +26,11 @@ WF_ATTN_AUTO = 0
 WF_ATTN_SINGLE = 1
 WF_ATTN_PAIR = 2
 
+# epilogues of wf_linear
+WF_EPI_STORE = 0
+WF_EPI_GELU_TANH = 1
+WF_EPI_GATED_RESIDUAL = 2
+
 # Every function include/wf.h declares: name -> (restype, argtypes)
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -50,6 +55,9 @@ SIGNATURES = {
     "wf_quantize_q_fp8": (_I, [_P, _P, _P, _P, _P]),
     "wf_quantize_k_fp8": (_I, [_P, _L, _I, _P, _P, _P, _P]),
     "wf_chunk_causal_attn_fp8qk": (_I, [_P, _L, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "wf_linear": (_I, [_P, _I, _I, _I, _P, _P, _P, _I, _P, _P, _I, _P, _P]),
+    "wf_qkv_proj_norm_rope_append": (_I, [_P, _L, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "wf_layer_norm_modulate": (_I, [_P, _I, _I, _P, _P, _P, _I, _P, _P]),
 }
 
 _lib = None
@@ -216,6 +224,34 @@ def wf_chunk_causal_attn_fp8qk(plan: Plan, round_: int, q8, q_scale, k8_cache, k
                                              _ptr(k8_cache), _ptr(k_scale), _ptr(v_cache),
                                              _ptr(o), _ptr(lse), _stream(stream)),
            "wf_chunk_causal_attn_fp8qk")
+
+
+def wf_linear(plan: Plan, x, w, y, bias=None, epilogue=WF_EPI_STORE, gate=None, resid=None,
+              rows_per_group=1, stream=None) -> None:
+    """y [M,N] = epilogue(x [M,K] @ w[N,K]^T + bias), bf16 in and out (see wf.h)."""
+    M, K = x.shape
+    N = w.shape[0]
+    _check(load().wf_linear(plan.handle, M, N, K, _ptr(x), _ptr(w), _ptr(bias), epilogue,
+                            _ptr(gate), _ptr(resid), rows_per_group, _ptr(y), _stream(stream)),
+           "wf_linear")
+
+
+def wf_qkv_proj_norm_rope_append(plan: Plan, round_: int, x, w_qkv, b_qkv, gamma_q, gamma_k,
+                                 q_out, k_cache, v_cache, stream=None) -> None:
+    """x [T,hidden] @ w_qkv[3HD,hidden]^T + b_qkv, then the append's norm/RoPE/ring write."""
+    _check(load().wf_qkv_proj_norm_rope_append(plan.handle, round_, x.shape[1], _ptr(x),
+                                               _ptr(w_qkv), _ptr(b_qkv), _ptr(gamma_q),
+                                               _ptr(gamma_k), _ptr(q_out), _ptr(k_cache),
+                                               _ptr(v_cache), _stream(stream)),
+           "wf_qkv_proj_norm_rope_append")
+
+
+def wf_layer_norm_modulate(plan: Plan, x, shift, scale, rows_per_group, y, stream=None) -> None:
+    """y = LayerNorm(x) * (1 + scale[g]) + shift[g], g = row // rows_per_group."""
+    M, C = x.shape
+    _check(load().wf_layer_norm_modulate(plan.handle, M, C, _ptr(x), _ptr(shift), _ptr(scale),
+                                         rows_per_group, _ptr(y), _stream(stream)),
+           "wf_layer_norm_modulate")
 
 
 def wf_sync_status(plan: Plan, stream=None) -> int:

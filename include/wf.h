@@ -194,6 +194,64 @@ WF_API int wf_chunk_causal_attn_fp8qk(wf_plan_t plan, long round, const void *q8
                                       const float *k_scale, const void *v_cache, void *o,
                                       float *lse, void *stream);
 
+/* ---- The DiT block around the wave round ---------------------------------
+ * "Wave Forcing" (abstract) runs every wave chunk through the layers of
+ * Wan2.1-T2V-1.3B in one forward pass.  Around the chunk-causal attention a DiT
+ * block holds dense projections (QKV, output, two feed-forward layers) and the
+ * adaLN-modulated LayerNorms before the attention and the feed-forward.  The
+ * pages print no formula for these layers; the definitions below are the plain
+ * ones.  Every chunk of a wave sits at its own denoising step, so modulation
+ * rows are per chunk: row n uses row n / rows_per_group of a modulation table.
+ *
+ * GEMMs are bf16 tensor-core products with fp32 accumulation, computed as
+ * y = x W^T with x [M][K] and W [N][K] (a linear layer's weight, out x in),
+ * both row-major bf16; the epilogue works in fp32 and rounds once to bf16.
+ * Each GEMM is one persistent kernel launch on `stream` (clusters of two CTAs).
+ * They use the plan only for its device status word and wait limit; calls on
+ * one plan must not run concurrently on the GPU. */
+
+enum {
+    WF_EPI_STORE = 0,            /* y = x W^T + bias                                   */
+    WF_EPI_GELU_TANH = 1,        /* y = gelu(x W^T + bias), tanh form of GELU          */
+    WF_EPI_GATED_RESIDUAL = 2    /* y = resid + gate[n / rows_per_group] * (x W^T + bias) */
+};
+
+/* A linear layer with a fused epilogue.  M >= 0 rows, N >= 32 and N % 32 == 0
+ * outputs, K >= 8 and K % 8 == 0 inputs.  x [M][K], w [N][K], y [M][N], resid
+ * [M][N]: bf16 device pointers, 16-byte aligned; bias [N] fp32 or NULL; gate [G][N]
+ * fp32 with G >= ceil(M / rows_per_group) (gated residual only; NULL otherwise).
+ * y must not overlap x or w (it may be resid).  M = 0 is a no-op that reads no
+ * pointer (they may be NULL).  Returns WF_ERR_INVALID_ARG on a bad size,
+ * epilogue, pointer or alignment. */
+WF_API int wf_linear(wf_plan_t plan, int M, int N, int K, const void *x, const void *w,
+                     const float *bias, int epilogue, const float *gate, const void *resid,
+                     int rows_per_group, void *y, void *stream);
+
+/* The QKV projection of the wave with wf_qk_norm_rope_append fused into its
+ * epilogue: y = x W_qkv^T + b_qkv ([T][3*H*D], q | k | v, each head-major), then
+ * per head the RMSNorm (gain gamma) and 3D RoPE of q and k, computed on the fp32
+ * accumulator (no rounding before the norm), and one rounding to bf16 each.  q
+ * goes to q_out [T][H][D]; k and v of wave chunk c go to ring slot (round + c)
+ * mod R of k_cache / v_cache, exactly where wf_qk_norm_rope_append writes them.
+ * x [T][hidden] and w_qkv [3*H*D][hidden] bf16 (hidden % 8 == 0), b_qkv [3*H*D]
+ * fp32 or NULL, gammas [H][D] fp32; device pointers, 16-byte aligned.  Positions
+ * are derived from the plan's grid (wf_plan_set_rope is required;
+ * WF_ERR_INVALID_ARG without it).  H*D must be a multiple of 128, and the
+ * rotation tables (W*F*dt/2 + grid_h*dh/2 + grid_w*dw/2 entries) must fit 3072
+ * entries; WF_ERR_UNSUPPORTED otherwise.  One kernel launch on `stream`. */
+WF_API int wf_qkv_proj_norm_rope_append(wf_plan_t plan, long round, int hidden, const void *x,
+                                        const void *w_qkv, const float *b_qkv,
+                                        const float *gamma_q, const float *gamma_k, void *q_out,
+                                        void *k_cache, void *v_cache, void *stream);
+
+/* LayerNorm over the last axis without a learned affine (eps 1e-6), then the
+ * adaLN modulation y = x_hat * (1 + scale[g]) + shift[g], g = n / rows_per_group.
+ * x, y [M][C] bf16; shift, scale [G][C] fp32; device pointers, 16-byte aligned;
+ * C % 8 == 0 and C <= 6144 (WF_ERR_UNSUPPORTED above).  y may equal x.  fp32
+ * arithmetic, one rounding to bf16.  One kernel launch on `stream`. */
+WF_API int wf_layer_norm_modulate(wf_plan_t plan, int M, int C, const void *x, const float *shift,
+                                  const float *scale, int rows_per_group, void *y, void *stream);
+
 /* Wait for `stream`, then read and clear the plan's device status word.
  * Returns WF_OK, WF_ERR_TIMEOUT (a bounded device wait expired) or WF_ERR_CUDA. */
 WF_API int wf_sync_status(wf_plan_t plan, void *stream);

@@ -178,3 +178,50 @@ def test_status_strings(wf):
     assert wf.status_string(0) == "ok"
     assert "timed out" in wf.status_string(wf.WF_ERR_TIMEOUT)
     assert wf.status_string(999) == "unknown status"
+
+
+def test_block_calls_validate_before_the_device(wf):
+    """wf_linear, wf_qkv_proj_norm_rope_append and wf_layer_norm_modulate: sizes,
+    epilogue codes, NULL and misaligned pointers, a missing RoPE grid and shapes the
+    kernels do not cover are reported before any device access; valid calls on a
+    machine without a GPU report WF_ERR_NO_DEVICE."""
+    import torch
+    lib = wf.load()
+    f = 1 << 20
+    p = wf.Plan(32, 1, 0, 1, 64)
+    E = wf.WF_ERR_INVALID_ARG
+    lin = lib.wf_linear
+    assert lin(p.handle, 10, 48, 64, f, f, None, 0, None, None, 1, f, None) == E   # N % 32
+    assert lin(p.handle, 10, 64, 60, f, f, None, 0, None, None, 1, f, None) == E   # K % 8
+    assert lin(p.handle, -1, 64, 64, f, f, None, 0, None, None, 1, f, None) == E
+    assert lin(p.handle, 10, 64, 64, f, f, None, 3, None, None, 1, f, None) == E   # epilogue
+    assert lin(p.handle, 10, 64, 64, f + 8, f, None, 0, None, None, 1, f, None) == E
+    assert lin(p.handle, 10, 64, 64, f, f, f + 4, 0, None, None, 1, f, None) == E  # bias align
+    assert lin(p.handle, 10, 64, 64, f, f, None, 2, None, f, 1, f, None) == E      # no gate
+    assert lin(p.handle, 10, 64, 64, f, f, None, 2, f, f, 0, f, None) == E         # rows/group
+    qkv = lib.wf_qkv_proj_norm_rope_append
+    pg = wf.Plan(300, 3, 1, 2, 128)                       # no grid set yet
+    assert qkv(pg.handle, 0, 256, f, f, None, f, f, f, f, f, None) == E
+    pg.set_rope(2, 6, 25)
+    assert qkv(pg.handle, 0, 250, f, f, None, f, f, f, f, f, None) == E             # hidden % 8
+    assert qkv(pg.handle, -1, 256, f, f, None, f, f, f, f, f, None) == E
+    assert qkv(pg.handle, 0, 256, f, f, None, f, None, f, f, f, None) == E
+    p1 = wf.Plan(64, 2, 0, 1, 64).set_rope(1, 8, 8)      # H*D = 64: not a multiple of 128
+    assert qkv(p1.handle, 0, 64, f, f, None, f, f, f, f, f, None) == wf.WF_ERR_UNSUPPORTED
+    big = wf.Plan(64 * 64, 1, 0, 2, 64).set_rope(1, 64, 64)   # 12 + 640 + 640 entries: fits
+    wide = wf.Plan(1 * 4000, 1, 0, 2, 64).set_rope(1, 1, 4000)  # w table 4000 * 5 > 3072
+    assert qkv(wide.handle, 0, 64, f, f, None, f, f, f, f, f, None) == wf.WF_ERR_UNSUPPORTED
+    ln = lib.wf_layer_norm_modulate
+    assert ln(p.handle, 10, 12, f, f, f, 1, f, None) == E                          # C % 8
+    assert ln(p.handle, 10, 6152, f, f, f, 1, f, None) == wf.WF_ERR_UNSUPPORTED
+    assert ln(p.handle, 10, 64, f, f, f, 0, f, None) == E
+    assert ln(p.handle, 10, 64, f, f + 4, f, 1, f, None) == E
+    if not torch.cuda.is_available():
+        N = wf.WF_ERR_NO_DEVICE
+        assert lin(p.handle, 10, 64, 64, f, f, None, 0, None, None, 1, f, None) == N
+        assert lin(p.handle, 10, 64, 64, f, f, f, 2, f, f, 3, f, None) == N
+        assert qkv(pg.handle, 0, 256, f, f, None, f, f, f, f, f, None) == N
+        assert qkv(big.handle, 0, 64, f, f, f, f, f, f, f, f, None) == N
+        assert ln(p.handle, 10, 64, f, f, f, 1, f, None) == N
+    for q in (p, pg, p1, big, wide):
+        q.destroy()
