@@ -326,6 +326,10 @@ def run_ours(args, rank, world, local):
     barrier(dist, dev)
 
     clk = clocks.summary(t_wall0, t_wall1)
+    block = None
+    if not args.no_block and not fp8 and w.H * w.D in wi.BLOCK_WIDTHS:
+        del q, k, v, x, hq, hk_, hv_, ho, pipe
+        block = run_block(args, plan, w, rnd, flops_step, dev, stream, peaks, dist)
     plan.destroy()
     if dist is not None:
         dist.destroy_process_group()
@@ -418,9 +422,122 @@ def run_ours(args, rank, world, local):
         "gpu_launches": (5 if fp8 else 2) * args.steps,
         "clocks": clk,
     }
+    if block is not None:
+        line["block"] = block
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
     return line
+
+
+def block_flops(w, hidden, ffn, attn_flops):
+    """Useful FLOPs of one DiT block over the wave: the four projections (QKV,
+    output, two feed-forward layers) plus the chunk-causal attention."""
+    HD = w.H * w.D
+    return 2.0 * w.T * (3 * HD * hidden + hidden * HD + 2 * hidden * ffn) + attn_flops
+
+
+def run_block(args, plan, w, r0, attn_flops, dev, stream, peaks, dist):
+    """One DiT block over the wave per step: LayerNorm + modulation, the QKV
+    projection with the norm/RoPE/ring append fused in, the chunk-causal
+    attention, the output projection with the gated residual, LayerNorm +
+    modulation, the GELU feed-forward layer and the second one with the gated
+    residual.  Random-init weights of the Wan block widths; per-chunk modulation
+    (each chunk sits at its own denoising step).  Device-timed with CUDA events
+    around every kernel; returns the "block" object of the JSON line."""
+    import torch
+    from chunk_causal_dit_b200 import wf
+
+    hidden, ffn = wi.BLOCK_WIDTHS[w.H * w.D]
+    b = wi.block_inputs(w, hidden, ffn, seed=0)
+    x = b.x.to(dev)
+    w_qkv, b_qkv = b.w_qkv.to(dev), b.b_qkv.to(dev)
+    w_o, b_o = b.w_o.to(dev), b.b_o.to(dev)
+    w_1, b_1 = b.w_1.to(dev), b.b_1.to(dev)
+    w_2, b_2 = b.w_2.to(dev), b.b_2.to(dev)
+    mod = b.mod.to(dev)
+    gq, gk = b.gamma_q.to(dev), b.gamma_k.to(dev)
+    h = torch.empty((w.T, hidden), dtype=torch.bfloat16, device=dev)
+    x1 = torch.empty_like(h)
+    x2 = torch.empty_like(h)
+    f = torch.empty((w.T, ffn), dtype=torch.bfloat16, device=dev)
+    q_out = torch.empty((w.T, w.H, w.D), dtype=torch.bfloat16, device=dev)
+    o = torch.empty_like(q_out)
+    kc = torch.zeros((w.R, w.L, w.H, w.D), dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros_like(kc)
+    o2 = o.view(w.T, w.H * w.D)
+    names = ["layer_norm_1", "qkv_norm_rope_append", "attention", "out_proj_gated",
+             "layer_norm_2", "ffn1_gelu", "ffn2_gated"]
+
+    def step(r, ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record(stream)
+        mark(0)
+        wf.wf_layer_norm_modulate(plan, x, mod[0], mod[1], w.L, h, stream)
+        mark(1)
+        wf.wf_qkv_proj_norm_rope_append(plan, r, h, w_qkv, b_qkv, gq, gk, q_out, kc, vc, stream)
+        mark(2)
+        wf.wf_chunk_causal_attn(plan, r, q_out, kc, vc, o, None, stream)
+        mark(3)
+        wf.wf_linear(plan, o2, w_o, x1, b_o, wf.WF_EPI_GATED_RESIDUAL, mod[2], x, w.L, stream)
+        mark(4)
+        wf.wf_layer_norm_modulate(plan, x1, mod[3], mod[4], w.L, h, stream)
+        mark(5)
+        wf.wf_linear(plan, h, w_1, f, b_1, wf.WF_EPI_GELU_TANH, None, None, 1, stream)
+        mark(6)
+        wf.wf_linear(plan, f, w_2, x2, b_2, wf.WF_EPI_GATED_RESIDUAL, mod[5], x1, w.L, stream)
+        mark(7)
+
+    rnd = r0
+    for _ in range(max(3, args.warmup)):
+        step(rnd)
+        rnd += 1
+    torch.cuda.synchronize(dev)
+    n = max(3, min(args.steps, 50))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(n)]
+    barrier(dist, dev)
+    torch.cuda.synchronize(dev)
+    for i in range(n):
+        step(rnd, evs[i])
+        rnd += 1
+    torch.cuda.synchronize(dev)
+    status = wf.wf_sync_status(plan, stream)
+    if status != wf.WF_OK:
+        raise SystemExit("block: device status %d (%s)" % (status, wf.status_string(status)))
+    per = {nm: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
+           for i, nm in enumerate(names)}
+    ms_step = allreduce_max(dist, statistics.mean(e[0].elapsed_time(e[7]) for e in evs), dev)
+    total = block_flops(w, hidden, ffn, attn_flops)
+    HD = w.H * w.D
+    gemm_flops = {"qkv_norm_rope_append": 2.0 * w.T * 3 * HD * hidden,
+                  "out_proj_gated": 2.0 * w.T * hidden * HD,
+                  "ffn1_gelu": 2.0 * w.T * hidden * ffn, "ffn2_gated": 2.0 * w.T * hidden * ffn}
+    peak_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    ln_bytes = 4.0 * w.T * hidden
+    tflops = total / (ms_step * 1e-3) / 1e12
+    return {
+        "what": "one DiT block over the wave (Wan %d/%d widths, random-init weights, per-chunk "
+                "modulation): LN, QKV + norm/RoPE/append, attention, out-proj + gated residual, "
+                "LN, FFN1 + GELU, FFN2 + gated residual" % (hidden, ffn),
+        "hidden": hidden, "ffn": ffn,
+        "steps": n,
+        "ms_per_step": round(ms_step, 4),
+        "useful_flop_per_step": total,
+        "tflops": round(tflops, 2),
+        "frac": round(tflops / peak_tf, 4),
+        "peak": peak_tf,
+        "chunks_per_s": round(w.n_wave / (ms_step * 1e-3), 2),
+        "ms_per_kernel": {k: round(v, 4) for k, v in per.items()},
+        "gemm_tflops": {k: round(fl / (per[k] * 1e-3) / 1e12, 1) for k, fl in gemm_flops.items()},
+        "gemm_frac": {k: round(fl / (per[k] * 1e-3) / 1e12 / peak_tf, 4)
+                      for k, fl in gemm_flops.items()},
+        "layer_norm_gbs": round(ln_bytes / (per["layer_norm_1"] * 1e-3) / 1e9, 1),
+        "layer_norm_frac": round(ln_bytes / (per["layer_norm_1"] * 1e-3) / 1e9 / hbm, 4),
+        "launches_per_step": 7,
+        "l2": l2_note((4 * w.T * hidden * 2 + w.T * ffn * 2 +
+                       2 * (4 * hidden * HD + 2 * hidden * ffn)) / 1e6),
+    }
 
 
 def run_round_loop(args, rank, world, local):
@@ -647,6 +764,8 @@ def main():
     ap.add_argument("--workload", default="wan13b_4step", choices=sorted(wi.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-block", action="store_true",
+                    help="skip the DiT-block leg (timed after the attention step)")
     ap.add_argument("--attn", default="bf16", choices=["bf16", "fp8qk"],
                     help="attention variant: bf16 (default) or E4M3 Q.K^T with bf16 P.V")
     ap.add_argument("--cpu-budget", type=float, default=12.0)

@@ -9,7 +9,9 @@
 //
 // HBM-bound: 2 bytes read and 2 written per element (the modulation tables are
 // small and stay in L1/L2).  One warp per row; lane l owns the 16-byte pieces
-// l, l + 32, ... of the row, all loaded before the reductions.
+// l, l + 32, ... of the row, all loaded before the reductions.  The kernel is
+// instantiated for a few counts of pieces per lane, so that a row of C channels
+// holds no more registers than it needs (occupancy sets the bytes in flight).
 #include <cuda_bf16.h>
 
 #include "sm100.cuh"
@@ -22,6 +24,7 @@ namespace {
 constexpr int kMaxPieces = 24;      // 16-byte pieces per lane: C <= 32 * 24 * 8 = 6144
 constexpr int kRowsPerBlock = 8;
 
+template <int kPer>
 __global__ void __launch_bounds__(32 * kRowsPerBlock)
 layer_norm_modulate_kernel(const uint16_t *__restrict__ x, const float *__restrict__ shift,
                            const float *__restrict__ scale, uint16_t *__restrict__ y, long M, int C,
@@ -32,15 +35,15 @@ layer_norm_modulate_kernel(const uint16_t *__restrict__ x, const float *__restri
     if (row >= M) return;                   // whole warps leave together
     const int pieces = C / 8;
     const uint4 *src = reinterpret_cast<const uint4 *>(x + row * C);
-    uint4 w[kMaxPieces];
+    uint4 w[kPer];
 #pragma unroll
-    for (int i = 0; i < kMaxPieces; ++i) {
+    for (int i = 0; i < kPer; ++i) {
         const int j = lane + 32 * i;
         w[i] = j < pieces ? __ldcs(src + j) : make_uint4(0u, 0u, 0u, 0u);
     }
     float s = 0.0f;
 #pragma unroll
-    for (int i = 0; i < kMaxPieces; ++i) {
+    for (int i = 0; i < kPer; ++i) {
         const uint32_t u[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e)
@@ -51,7 +54,7 @@ layer_norm_modulate_kernel(const uint16_t *__restrict__ x, const float *__restri
     const float mean = s / static_cast<float>(C);
     float v = 0.0f;
 #pragma unroll
-    for (int i = 0; i < kMaxPieces; ++i) {
+    for (int i = 0; i < kPer; ++i) {
         if (lane + 32 * i >= pieces) break;
         const uint32_t u[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
 #pragma unroll
@@ -69,7 +72,7 @@ layer_norm_modulate_kernel(const uint16_t *__restrict__ x, const float *__restri
     const float4 *sc4 = reinterpret_cast<const float4 *>(scale + g * C);
     uint4 *dst = reinterpret_cast<uint4 *>(y + row * C);
 #pragma unroll
-    for (int i = 0; i < kMaxPieces; ++i) {
+    for (int i = 0; i < kPer; ++i) {
         const int j = lane + 32 * i;
         if (j >= pieces) break;
         const uint32_t u[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
@@ -99,8 +102,26 @@ cudaError_t launch_layer_norm_modulate(const uint16_t *x, const float *shift, co
 {
     if (M == 0) return cudaSuccess;
     const dim3 grid(static_cast<unsigned>((M + kRowsPerBlock - 1) / kRowsPerBlock));
-    layer_norm_modulate_kernel<<<grid, 32 * kRowsPerBlock, 0, stream>>>(x, shift, scale, y, M, C,
-                                                                        rows_per_group, eps);
+    const int per_lane = (C / 8 + 31) / 32;
+    auto go = [&](auto kern) {
+        kern<<<grid, 32 * kRowsPerBlock, 0, stream>>>(x, shift, scale, y, M, C, rows_per_group, eps);
+    };
+    if (per_lane <= 2)
+        go(layer_norm_modulate_kernel<2>);
+    else if (per_lane <= 4)
+        go(layer_norm_modulate_kernel<4>);
+    else if (per_lane <= 6)
+        go(layer_norm_modulate_kernel<6>);
+    else if (per_lane <= 8)
+        go(layer_norm_modulate_kernel<8>);
+    else if (per_lane <= 12)
+        go(layer_norm_modulate_kernel<12>);
+    else if (per_lane <= 16)
+        go(layer_norm_modulate_kernel<16>);
+    else if (per_lane <= 20)
+        go(layer_norm_modulate_kernel<20>);
+    else
+        go(layer_norm_modulate_kernel<kMaxPieces>);
     return cudaGetLastError();
 }
 

@@ -267,6 +267,15 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank)
     return r;
 }
 
+// arrive, with no memory ordering, on an mbarrier that may live in another CTA of
+// the cluster (for a signal that orders nothing but the arriving thread's own
+// completed work, e.g. TMEM loads already waited for)
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];"
+                 ::"r"(cluster_addr) : "memory");
+}
+
 // arrive on an mbarrier that may live in another CTA of the cluster
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
 {

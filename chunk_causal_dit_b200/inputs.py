@@ -135,6 +135,9 @@ def f32_vector(shape, scale: float, seed: int, stream: int, salt: int = 0) -> to
 # Hidden and feed-forward widths of the Wan2.1-T2V-1.3B block (12 heads x 128 = 1536).
 WAN13B_HIDDEN = 1536
 WAN13B_FFN = 8960
+# (hidden, feed-forward) widths of the block by attention width H*D: the 1.3B model
+# (12 x 128) and the 14B model (40 x 128).
+BLOCK_WIDTHS = {12 * 128: (WAN13B_HIDDEN, WAN13B_FFN), 40 * 128: (5120, 13824)}
 
 
 @dataclass
