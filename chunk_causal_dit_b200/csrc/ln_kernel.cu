@@ -8,10 +8,11 @@
 // fp32 arithmetic and one rounding to bf16.
 //
 // HBM-bound: 2 bytes read and 2 written per element (the modulation tables are
-// small and stay in L1/L2).  One warp per row; lane l owns the 16-byte pieces
-// l, l + 32, ... of the row, all loaded before the reductions.  The kernel is
-// instantiated for a few counts of pieces per lane, so that a row of C channels
-// holds no more registers than it needs (occupancy sets the bytes in flight).
+// small; each block stages its rows' group in shared memory).  One warp per
+// row; lane l owns the 16-byte pieces l, l + 32, ... of the row, all loaded
+// before the reductions.  The kernel is instantiated for a few counts of pieces
+// per lane, so that a row of C channels holds no more registers than it needs
+// (occupancy sets the bytes in flight).
 #include <cuda_bf16.h>
 
 #include "sm100.cuh"
@@ -30,17 +31,33 @@ layer_norm_modulate_kernel(const uint16_t *__restrict__ x, const float *__restri
                            const float *__restrict__ scale, uint16_t *__restrict__ y, long M, int C,
                            int rows_per_group, float eps)
 {
+    // shift and scale of the group of the block's first row, staged while the
+    // row loads are in flight (a block's rows straddle two groups only at a
+    // chunk boundary; such rows read their own group's rows from global memory)
+    extern __shared__ float4 s_mod[];            // [C/4] shift, then [C/4] scale
     const int lane = threadIdx.x & 31;
-    const long row = static_cast<long>(blockIdx.x) * kRowsPerBlock + (threadIdx.x >> 5);
-    if (row >= M) return;                   // whole warps leave together
+    const long row0 = static_cast<long>(blockIdx.x) * kRowsPerBlock;
+    const long row = row0 + (threadIdx.x >> 5);
+    const bool live = row < M;
     const int pieces = C / 8;
-    const uint4 *src = reinterpret_cast<const uint4 *>(x + row * C);
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + (live ? row : row0) * C);
     uint4 w[kPer];
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
         const int j = lane + 32 * i;
-        w[i] = j < pieces ? __ldcs(src + j) : make_uint4(0u, 0u, 0u, 0u);
+        w[i] = (live && j < pieces) ? __ldcs(src + j) : make_uint4(0u, 0u, 0u, 0u);
     }
+    const long g0 = row0 / rows_per_group;
+    {
+        const float4 *sh = reinterpret_cast<const float4 *>(shift + g0 * C);
+        const float4 *sc = reinterpret_cast<const float4 *>(scale + g0 * C);
+        for (int i = threadIdx.x; i < C / 4; i += 32 * kRowsPerBlock) {
+            s_mod[i] = __ldg(sh + i);
+            s_mod[C / 4 + i] = __ldg(sc + i);
+        }
+    }
+    __syncthreads();
+    if (!live) return;                      // whole warps leave together
     float s = 0.0f;
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
@@ -68,16 +85,16 @@ layer_norm_modulate_kernel(const uint16_t *__restrict__ x, const float *__restri
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
     const float rstd = rsqrtf(v / static_cast<float>(C) + eps);
     const long g = row / rows_per_group;
-    const float4 *sh4 = reinterpret_cast<const float4 *>(shift + g * C);
-    const float4 *sc4 = reinterpret_cast<const float4 *>(scale + g * C);
+    const float4 *sh4 = g == g0 ? s_mod : reinterpret_cast<const float4 *>(shift + g * C);
+    const float4 *sc4 = g == g0 ? s_mod + C / 4 : reinterpret_cast<const float4 *>(scale + g * C);
     uint4 *dst = reinterpret_cast<uint4 *>(y + row * C);
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
         const int j = lane + 32 * i;
         if (j >= pieces) break;
         const uint32_t u[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
-        const float4 sa = __ldg(sh4 + 2 * j), sb = __ldg(sh4 + 2 * j + 1);
-        const float4 ca = __ldg(sc4 + 2 * j), cb = __ldg(sc4 + 2 * j + 1);
+        const float4 sa = sh4[2 * j], sb = sh4[2 * j + 1];
+        const float4 ca = sc4[2 * j], cb = sc4[2 * j + 1];
         const float shv[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
         const float scv[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
         uint32_t o[4];
@@ -104,7 +121,8 @@ cudaError_t launch_layer_norm_modulate(const uint16_t *x, const float *shift, co
     const dim3 grid(static_cast<unsigned>((M + kRowsPerBlock - 1) / kRowsPerBlock));
     const int per_lane = (C / 8 + 31) / 32;
     auto go = [&](auto kern) {
-        kern<<<grid, 32 * kRowsPerBlock, 0, stream>>>(x, shift, scale, y, M, C, rows_per_group, eps);
+        kern<<<grid, 32 * kRowsPerBlock, 2 * C * sizeof(float), stream>>>(x, shift, scale, y, M,
+                                                                           C, rows_per_group, eps);
     };
     if (per_lane <= 2)
         go(layer_norm_modulate_kernel<2>);
