@@ -540,6 +540,173 @@ def run_block(args, plan, w, r0, attn_flops, dev, stream, peaks, dist):
     }
 
 
+# Peer-to-peer copy bandwidth per direction between two B200s over NVLink 5, as
+# measured (900 GB/s nominal).
+PEER_COPY_GBS = 770.0
+
+
+def run_wp(args, rank, world, local):
+    """Wave Parallelism (chunk_causal_dit_b200.wave_parallel): the wave's chunks split
+    over ranks; one step is one layer of one round (append, one-way K/V delivery,
+    attention), the round advancing every step.
+
+    Under torchrun every rank is a GPU and the delivery is NCCL point-to-point; the
+    step time is the device-timed max over ranks, and `value` is the whole wave's
+    useful TFLOP/s (strong scaling).  In one process with --wp N > 1 the N ranks'
+    kernels run one after another on the one GPU (device copies stand in for the
+    delivery and are not timed); the line then reports each rank's kernel times
+    and a step time *projected* as the slowest rank's append + attention plus the
+    delivery of its incoming K/V at the peer-copy bandwidth, next to the
+    single-GPU round measured in the same process."""
+    import torch
+    from chunk_causal_dit_b200 import wf
+    from chunk_causal_dit_b200.wave_parallel import LibwfKernels, WaveParallelRound
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = make_group(world, "nccl")
+    w = wi.WORKLOADS[args.workload]
+    emulate = world == 1
+    n_ranks = args.wp if emulate else world
+    if not 1 <= n_ranks <= w.n_wave:
+        raise SystemExit("Wave Parallelism needs 1..%d ranks (one wave chunk each at least)"
+                         % w.n_wave)
+    x = wi.wave_inputs(w, seed=0)
+    hk, hv = wi.history_prefill(w, seed=0)
+    gq, gk = x.gamma_q.to(dev), x.gamma_k.to(dev)
+    kern = LibwfKernels(gq, gk)
+    r0 = w.n_hist
+    mine = list(range(n_ranks)) if emulate else [rank]
+    wps, ten = {}, {}
+    for k in mine:
+        kw = {"world": n_ranks, "rank": k} if emulate else {}
+        wp = WaveParallelRound(w.L, w.n_wave, w.n_hist, w.H, w.D, (w.F, w.gh, w.gw), kern, **kw)
+        rows = slice(wp.c0 * w.L, wp.c1 * w.L)
+        t = {"q": x.q[rows].to(dev), "k": x.k[rows].to(dev), "v": x.v[rows].to(dev)}
+        t["q_out"] = torch.empty_like(t["q"])
+        t["o"] = torch.empty_like(t["q"])
+        t["kc"] = torch.empty(wp.ring_shape(), dtype=torch.bfloat16, device=dev)
+        t["vc"] = torch.empty_like(t["kc"])
+        wp.prefill_history(r0, [(r0 - w.n_hist + j, hk[j].to(dev), hv[j].to(dev))
+                                for j in range(w.n_hist)], t["kc"], t["vc"])
+        wps[k], ten[k] = wp, t
+    stream = torch.cuda.current_stream(dev)
+
+    def layer(r, ev=None):
+        if not emulate:
+            wp, t = wps[rank], ten[rank]
+            wp.run_layer(r, t["q"], t["k"], t["v"], t["q_out"], t["kc"], t["vc"], t["o"])
+            return
+        for i, k in enumerate(mine):
+            wp, t = wps[k], ten[k]
+            if ev is not None:
+                ev[i][0].record(stream)
+            kern.append(wp.plan, r + wp.c0, t["q"], t["k"], t["v"], t["q_out"], t["kc"], t["vc"])
+            if ev is not None:
+                ev[i][1].record(stream)
+        for k in mine:                       # stand-in for the NCCL delivery (not timed)
+            for src, g in wps[k].incoming(r):
+                ten[k]["kc"][wps[k].slot(g)].copy_(ten[src]["kc"][wps[src].slot(g)])
+                ten[k]["vc"][wps[k].slot(g)].copy_(ten[src]["vc"][wps[src].slot(g)])
+        for i, k in enumerate(mine):
+            wp, t = wps[k], ten[k]
+            if ev is not None:
+                ev[i][2].record(stream)
+            kern.attention(wp.plan, r + wp.c0, t["q_out"], t["kc"], t["vc"], t["o"])
+            if ev is not None:
+                ev[i][3].record(stream)
+
+    rnd = r0
+    for _ in range(args.warmup):
+        layer(rnd)
+        rnd += 1
+    torch.cuda.synchronize(dev)
+    full = wf.Plan(w.L, w.n_wave, w.n_hist, w.H, w.D)
+    flops_step = wf.wf_useful_flops(full, r0)
+    full.destroy()
+    steps = args.steps
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in mine]
+           for _ in range(steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dist, dev)
+    torch.cuda.synchronize(dev)
+    start.record(stream)
+    for i in range(steps):
+        layer(rnd, evs[i] if emulate else None)
+        rnd += 1
+    stop.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    for k in mine:
+        st = wf.wf_sync_status(wps[k].plan)
+        if st != wf.WF_OK:
+            raise SystemExit("wave parallel: device status %d (%s)" % (st, wf.status_string(st)))
+    ms_step = allreduce_max(dist, start.elapsed_time(stop), dev) / steps
+    line = None
+    if rank == 0:
+        chunk_bytes = 2 * w.L * w.H * w.D * 2            # K and V of one chunk, bf16
+        line = {
+            "metric": METRIC + " (Wave Parallelism, %d ranks)" % n_ranks,
+            "unit": "TFLOP/s", "n_gpus": world, "steps": steps, "warmup": args.warmup,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded bf16 N(0,1) q/k/v and history)",
+            "config": {"workload": w.name, "wave_parallel_ranks": n_ranks,
+                       "chunks_per_rank": [wp.n for wp in wps.values()] if emulate else None,
+                       "parallelism": "wave-parallel %d (one-way K/V delivery, NCCL p2p)"
+                       % n_ranks},
+        }
+        if not emulate:
+            line.update({"value": round(flops_step / (ms_step * 1e-3) / 1e12, 3),
+                         "ms_per_step": round(ms_step, 5), "projected": False})
+        else:
+            per = []
+            for i, k in enumerate(mine):
+                wp = wps[k]
+                app = statistics.mean(e[i][0].elapsed_time(e[i][1]) for e in evs)
+                att = statistics.mean(e[i][2].elapsed_time(e[i][3]) for e in evs)
+                recv = len(wp.incoming(r0)) * chunk_bytes
+                per.append({"rank": k, "chunks": [wp.c0, wp.c1], "append_ms": round(app, 5),
+                            "attention_ms": round(att, 5), "recv_bytes": recv,
+                            "recv_ms_at_peer_copy": round(recv / (PEER_COPY_GBS * 1e6), 5)})
+            proj = max(p["append_ms"] + p["recv_ms_at_peer_copy"] + p["attention_ms"]
+                       for p in per)
+            # the single-GPU round in the same process, for the comparison
+            plan = wf.Plan(w.L, w.n_wave, w.n_hist, w.H, w.D).set_rope(w.F, w.gh, w.gw)
+            q, k_, v = x.q.to(dev), x.k.to(dev), x.v.to(dev)
+            kc = torch.empty((w.R, w.L, w.H, w.D), dtype=torch.bfloat16, device=dev)
+            vc = torch.empty_like(kc)
+            q_out, o = torch.empty_like(q), torch.empty_like(q)
+            for _ in range(3):
+                wf.wf_qk_norm_rope_append(plan, r0, q, k_, v, None, gq, gk, q_out, kc, vc)
+                wf.wf_chunk_causal_attn(plan, r0, q_out, kc, vc, o)
+            torch.cuda.synchronize(dev)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for i in range(steps):
+                wf.wf_qk_norm_rope_append(plan, r0 + i, q, k_, v, None, gq, gk, q_out, kc, vc)
+                wf.wf_chunk_causal_attn(plan, r0 + i, q_out, kc, vc, o)
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            single = a.elapsed_time(b) / steps
+            plan.destroy()
+            line.update({
+                "value": round(flops_step / (proj * 1e-3) / 1e12, 3),
+                "ms_per_step": round(proj, 5), "projected": True,
+                "projection": "max over ranks of (append + incoming K/V at %.0f GB/s peer copy + "
+                              "attention), each rank's kernels timed alone on one B200"
+                              % PEER_COPY_GBS,
+                "per_rank": per,
+                "single_gpu_ms_per_step": round(single, 5),
+                "speedup_projected": round(single / proj, 3),
+                "emulation_ms_per_step": round(ms_step, 5),
+            })
+    for wp in wps.values():
+        wp.destroy()
+    if dist is not None:
+        dist.destroy_process_group()
+    return line
+
+
 def run_round_loop(args, rank, world, local):
     """Full rounds of a multi-layer workload: every round runs, layer after layer,
     the append and the attention of each layer on that layer's own ring, then
@@ -768,6 +935,9 @@ def main():
                     help="skip the DiT-block leg (timed after the attention step)")
     ap.add_argument("--attn", default="bf16", choices=["bf16", "fp8qk"],
                     help="attention variant: bf16 (default) or E4M3 Q.K^T with bf16 P.V")
+    ap.add_argument("--wp", type=int, default=0,
+                    help="Wave Parallelism: under torchrun, split the wave over the ranks; "
+                         "in one process, emulate N ranks on the one GPU (projected time)")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--ref-pairs", type=int, default=48)
     args = ap.parse_args()
@@ -778,6 +948,8 @@ def main():
     rank, world, local = dist_setup(args.gpus)
     if args.impl == "reference":
         line = run_reference(args, rank, world)
+    elif args.wp:
+        line = run_wp(args, rank, world, local)
     elif wi.WORKLOADS[args.workload].layers > 1:
         line = run_round_loop(args, rank, world, local)
     else:
