@@ -398,6 +398,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
             tma_prefetch_desc(&tmap_a);
             tma_prefetch_desc(&tmap_b);
             uint32_t it = 0;
+            const bool withheld = p.withhold != 0;   // test hook: stage 0's first fill never comes
             bool ok = true;
             for (int t = cid; ok && t < p.n_tiles; t += ncl) {
                 const int mb = t / p.n_ntiles, nb = t - mb * p.n_ntiles;
@@ -408,6 +409,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                     if (!(ok = wait_bar(bar(B::empty + st), ((it / kStages) & 1u) ^ 1u, ctl,
                                         kWhereProducer)))
                         break;
+                    if (withheld && it == 0) continue;
                     if (leader) mbar_arrive_expect_tx(bar(B::full + st), 2 * kStageBytes);
                     const uint32_t dst = sbase + st * kStageBytes;
                     tma_load_2d_pair(dst, &tmap_a, lead(B::full + st), kb * BK, arow);
@@ -415,8 +417,10 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                 }
             }
             if (!ok && leader) {
-                // both CTAs' copies complete on the leader's barriers: let them land
-                for (uint32_t s = 0; s < static_cast<uint32_t>(kStages); ++s) {
+                // both CTAs' copies complete on the leader's barriers: let the armed
+                // fills land.  With the first fill of stage 0 withheld, stage 0 was
+                // never filled (its next fill waits for a consumption that never came).
+                for (uint32_t s = withheld ? 1u : 0u; s < static_cast<uint32_t>(kStages); ++s) {
                     const uint32_t fills = (it + kStages - 1 - s) / kStages;
                     if (fills)
                         wait_bar(bar(B::full + s), (fills - 1) & 1u, ctl, kWhereDrain, true);

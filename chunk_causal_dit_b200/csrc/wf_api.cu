@@ -476,6 +476,7 @@ int wf_linear(wf_plan_t p, int M, int N, int K, const void *x, const void *w, co
     g.gate = gate;
     g.rows_per_group = rows_per_group < 1 ? 1 : rows_per_group;
     g.wait_limit = p->wait_limit;
+    g.withhold = p->withhold_q;
     g.words = p->words;
     CUtensorMap ma, mb;
     if (!encode_map_2d(&ma, x, M, K) || !encode_map_2d(&mb, w, N, K)) return WF_ERR_CUDA;
@@ -525,6 +526,7 @@ int wf_qkv_proj_norm_rope_append(wf_plan_t p, long round, int hidden, const void
     g.rope = p->rope;
     g.n_tab = static_cast<int>(n_tab);
     g.wait_limit = p->wait_limit;
+    g.withhold = p->withhold_q;
     g.words = p->words;
     CUtensorMap ma, mb;
     if (!encode_map_2d(&ma, x, T, hidden) || !encode_map_2d(&mb, w_qkv, g.N, hidden))

@@ -110,6 +110,7 @@ struct GemmParams {
     RopeParams rope;
     int n_tab;                // (cos, sin) table entries: W*F*dt/2 + gh*dh/2 + gw*dw/2
     unsigned long long wait_limit;
+    int withhold;             // test hook: no CTA issues (or arms) its first stage's copies
     DeviceWords *words;
 };
 

@@ -88,8 +88,9 @@ WF_API int wf_plan_set_rope_split(wf_plan_t plan, int d_t, int d_h, int d_w);
 /* RMSNorm epsilon (>= 0). */
 WF_API int wf_plan_set_norm_eps(wf_plan_t plan, double eps);
 
-/* Device-wait limit in SM clock cycles for the attention kernel (0 = default,
- * about two seconds).  Exposed so that tests can make a wait expire quickly. */
+/* Device-wait limit in SM clock cycles for the attention and GEMM kernels
+ * (0 = default, about two seconds).  Exposed so that tests can make a wait
+ * expire quickly. */
 WF_API int wf_plan_set_wait_limit(wf_plan_t plan, unsigned long long cycles);
 
 /* Test hook for failure detection, off by default.  With on != 0 the attention
@@ -98,7 +99,10 @@ WF_API int wf_plan_set_wait_limit(wf_plan_t plan, unsigned long long cycles);
  * warp's wait for it cannot complete: the bounded wait expires, the kernel
  * stops cleanly (copies and MMAs in flight drained, TMEM freed) and
  * wf_sync_status returns WF_ERR_TIMEOUT.  Nothing faults or traps; the
- * context stays usable.  Pair it with a short wf_plan_set_wait_limit. */
+ * context stays usable.  Pair it with a short wf_plan_set_wait_limit.  The
+ * GEMM calls (wf_linear, wf_qkv_proj_norm_rope_append) honour the same hook:
+ * no CTA issues, and the leader does not arm, the copies of the first K slice,
+ * so the MMA's wait for it expires the same way. */
 WF_API int wf_plan_set_withhold_q(wf_plan_t plan, int on);
 
 /* Attention kernel variant.  Both compute the same result (within the

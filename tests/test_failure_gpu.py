@@ -54,3 +54,47 @@ def test_expired_wait_reports_timeout_and_context_survives(wf, kind):
     ref, _ = oracle.round_attention(cache, r, W, Hh, wi.bits(q.cpu()), rows, heads)
     assert_attention_close(o.float().cpu().numpy().reshape(-1, D), ref, "after timeout")
     plan.destroy()
+
+
+@pytest.mark.parametrize("call", ["linear", "qkv"])
+def test_gemm_expired_wait_reports_timeout_and_context_survives(wf, call):
+    """The CTA-pair GEMM's bounded waits: with the first K slice withheld the
+    MMA's wait expires, both CTAs stop (copies drained, TMEM freed) and the call
+    reports WF_ERR_TIMEOUT; the next call on the same plan is correct."""
+    import oracle.block as ob
+    dev = "cuda"
+    F, gh, gw, W, Hh, H, D, C = 2, 6, 25, 3, 1, 2, 128, 256
+    L, T = F * gh * gw, W * F * gh * gw
+    x = wi.bf16_normal((T, C), 4, wi.STREAM_X)
+    w_qkv = wi.bf16_weight(3 * H * D, C, 4)
+    gq, gk = wi.gains(H, D, 4)
+    plan = wf.Plan(L, W, Hh, H, D).set_rope(F, gh, gw)
+    q_out = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+    kc = torch.zeros((W + Hh, L, H, D), dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros_like(kc)
+    y = torch.empty((T, 3 * H * D), dtype=torch.bfloat16, device=dev)
+
+    def run():
+        if call == "linear":
+            wf.wf_linear(plan, x.to(dev), w_qkv.to(dev), y)
+        else:
+            wf.wf_qkv_proj_norm_rope_append(plan, 1, x.to(dev), w_qkv.to(dev), None,
+                                            gq.to(dev), gk.to(dev), q_out, kc, vc)
+
+    plan.set_wait_limit(1 << 24).set_withhold_q(True)     # ~10 ms of SM clock
+    run()
+    assert wf.wf_sync_status(plan) == wf.WF_ERR_TIMEOUT
+    assert wf.wf_sync_status(plan) == wf.WF_OK
+    plan.set_withhold_q(False).set_wait_limit(0)
+    run()
+    torch.cuda.synchronize()
+    assert wf.wf_sync_status(plan) == wf.WF_OK
+    ref = ob.linear_f64(wi.bits(x), wi.bits(w_qkv))
+    if call == "linear":
+        got = y.float().cpu().numpy()
+    else:   # v is the projection itself, rounded once
+        got = torch.cat([vc[(1 + c) % (W + Hh)] for c in range(W)]).float().cpu().numpy()
+        got = got.reshape(T, H * D)
+        ref = ref[:, 2 * H * D:]
+    assert np.abs(got - ref).max() <= 2.0 ** -6     # bf16 rounding of values up to ~4
+    plan.destroy()
