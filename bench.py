@@ -327,9 +327,9 @@ def run_ours(args, rank, world, local):
 
     clk = clocks.summary(t_wall0, t_wall1)
     block = None
-    if not args.no_block and not fp8 and w.H * w.D in wi.BLOCK_WIDTHS:
+    if not args.no_block and w.H * w.D in wi.BLOCK_WIDTHS:
         del q, k, v, x, hq, hk_, hv_, ho, pipe
-        block = run_block(args, plan, w, rnd, flops_step, dev, stream, peaks, dist)
+        block = run_block(args, plan, w, rnd, flops_step, dev, stream, peaks, dist, fp8)
     plan.destroy()
     if dist is not None:
         dist.destroy_process_group()
@@ -436,7 +436,7 @@ def block_flops(w, hidden, ffn, attn_flops):
     return 2.0 * w.T * (3 * HD * hidden + hidden * HD + 2 * hidden * ffn) + attn_flops
 
 
-def run_block(args, plan, w, r0, attn_flops, dev, stream, peaks, dist):
+def run_block(args, plan, w, r0, attn_flops, dev, stream, peaks, dist, fp8=False):
     """One DiT block over the wave per step: LayerNorm + modulation, the QKV
     projection with the norm/RoPE/ring append fused in, the chunk-causal
     attention, the output projection with the gated residual, LayerNorm +
@@ -467,6 +467,16 @@ def run_block(args, plan, w, r0, attn_flops, dev, stream, peaks, dist):
     o2 = o.view(w.T, w.H * w.D)
     names = ["layer_norm_1", "qkv_norm_rope_append", "attention", "out_proj_gated",
              "layer_norm_2", "ffn1_gelu", "ffn2_gated"]
+    if fp8:
+        # E4M3 q (per row) and key ring (per 128-row tile); every slot is quantized
+        # once here, later history chunks in the round that appended them
+        nt = (w.L + 127) // 128
+        q8 = torch.empty((w.T, w.H, w.D), dtype=torch.uint8, device=dev)
+        q_scale = torch.empty((w.H, w.T), dtype=torch.float32, device=dev)
+        k8 = torch.empty((w.R, w.L, w.H, w.D), dtype=torch.uint8, device=dev)
+        k_scale = torch.empty((w.R, nt, w.H), dtype=torch.float32, device=dev)
+        wf.wf_quantize_k_fp8(plan, r0 - w.n_hist, w.R, kc, k8, k_scale, stream)
+        names[2] = "attention_fp8qk (with the q and k quantization)"
 
     def step(r, ev=None):
         def mark(i):
@@ -477,7 +487,12 @@ def run_block(args, plan, w, r0, attn_flops, dev, stream, peaks, dist):
         mark(1)
         wf.wf_qkv_proj_norm_rope_append(plan, r, h, w_qkv, b_qkv, gq, gk, q_out, kc, vc, stream)
         mark(2)
-        wf.wf_chunk_causal_attn(plan, r, q_out, kc, vc, o, None, stream)
+        if fp8:
+            wf.wf_quantize_q_fp8(plan, q_out, q8, q_scale, stream)
+            wf.wf_quantize_k_fp8(plan, r, w.n_wave, kc, k8, k_scale, stream)
+            wf.wf_chunk_causal_attn_fp8qk(plan, r, q8, q_scale, k8, k_scale, vc, o, None, stream)
+        else:
+            wf.wf_chunk_causal_attn(plan, r, q_out, kc, vc, o, None, stream)
         mark(3)
         wf.wf_linear(plan, o2, w_o, x1, b_o, wf.WF_EPI_GATED_RESIDUAL, mod[2], x, w.L, stream)
         mark(4)
@@ -509,6 +524,8 @@ def run_block(args, plan, w, r0, attn_flops, dev, stream, peaks, dist):
     ms_step = allreduce_max(dist, statistics.mean(e[0].elapsed_time(e[7]) for e in evs), dev)
     total = block_flops(w, hidden, ffn, attn_flops)
     HD = w.H * w.D
+    if fp8:
+        per["attention"] = per.pop(names[2])
     gemm_flops = {"qkv_norm_rope_append": 2.0 * w.T * 3 * HD * hidden,
                   "out_proj_gated": 2.0 * w.T * hidden * HD,
                   "ffn1_gelu": 2.0 * w.T * hidden * ffn, "ffn2_gated": 2.0 * w.T * hidden * ffn}
@@ -534,7 +551,9 @@ def run_block(args, plan, w, r0, attn_flops, dev, stream, peaks, dist):
                       for k, fl in gemm_flops.items()},
         "layer_norm_gbs": round(ln_bytes / (per["layer_norm_1"] * 1e-3) / 1e9, 1),
         "layer_norm_frac": round(ln_bytes / (per["layer_norm_1"] * 1e-3) / 1e9 / hbm, 4),
-        "launches_per_step": 7,
+        "attention": "fp8qk (E4M3 Q.K^T, bf16 P.V; q and k quantization included)" if fp8
+                     else "bf16",
+        "launches_per_step": 9 if fp8 else 7,
         "l2": l2_note((4 * w.T * hidden * 2 + w.T * ffn * 2 +
                        2 * (4 * hidden * HD + 2 * hidden * ffn)) / 1e6),
     }
