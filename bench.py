@@ -726,6 +726,120 @@ def run_wp(args, rank, world, local):
     return line
 
 
+def run_block_round_loop(args, rank, world, local):
+    """Full rounds of the model's blocks: every round runs the DiT block (the
+    "block" leg of run_ours) of each of the workload's layers, layer after layer,
+    the residual stream flowing from one layer into the next, each layer with its
+    own ring and its own random-init weights; the rings advance one chunk per
+    round.  Reports per-round latency (median, p90), rounds/s (one output chunk
+    per round after pipeline fill) and useful TFLOP/s of the round."""
+    import torch
+    from chunk_causal_dit_b200 import wf
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = make_group(world, "nccl")
+    w = wi.WORKLOADS[args.workload]
+    if w.H * w.D not in wi.BLOCK_WIDTHS:
+        raise SystemExit("no block widths for %d x %d heads" % (w.H, w.D))
+    hidden, ffn = wi.BLOCK_WIDTHS[w.H * w.D]
+    peaks, _ = load_peaks()
+    plan = wf.Plan(w.L, w.n_wave, w.n_hist, w.H, w.D).set_rope(w.F, w.gh, w.gw)
+    layers = [wi.block_weights_on(dev, w, hidden, ffn, rank, l) for l in range(w.layers)]
+    g = torch.Generator(device=dev)
+    g.manual_seed(1009 * rank + 7)
+    rings = [tuple(torch.randn((w.R, w.L, w.H, w.D), generator=g, device=dev).to(torch.bfloat16)
+                   for _ in range(2)) for _ in range(w.layers)]
+    x0 = wi.bf16_normal((w.T, hidden), rank, wi.STREAM_X).to(dev)
+    X = torch.empty_like(x0)          # the residual stream, updated in place layer by layer
+    h = torch.empty_like(x0)
+    f = torch.empty((w.T, ffn), dtype=torch.bfloat16, device=dev)
+    q_out = torch.empty((w.T, w.H, w.D), dtype=torch.bfloat16, device=dev)
+    o = torch.empty_like(q_out)
+    o2 = o.view(w.T, w.H * w.D)
+    stream = torch.cuda.current_stream(dev)
+    r0 = w.n_hist
+
+    def run_round(r):
+        X.copy_(x0)
+        for lw, (kc, vc) in zip(layers, rings):
+            mod = lw["mod"]
+            wf.wf_layer_norm_modulate(plan, X, mod[0], mod[1], w.L, h, stream)
+            wf.wf_qkv_proj_norm_rope_append(plan, r, h, lw["w_qkv"], lw["b_qkv"], lw["gamma_q"],
+                                            lw["gamma_k"], q_out, kc, vc, stream)
+            wf.wf_chunk_causal_attn(plan, r, q_out, kc, vc, o, None, stream)
+            # gated residuals in place: X = X + gate * (...)
+            wf.wf_linear(plan, o2, lw["w_o"], X, lw["b_o"], wf.WF_EPI_GATED_RESIDUAL, mod[2], X,
+                         w.L, stream)
+            wf.wf_layer_norm_modulate(plan, X, mod[3], mod[4], w.L, h, stream)
+            wf.wf_linear(plan, h, lw["w_1"], f, lw["b_1"], wf.WF_EPI_GELU_TANH, None, None, 1,
+                         stream)
+            wf.wf_linear(plan, f, lw["w_2"], X, lw["b_2"], wf.WF_EPI_GATED_RESIDUAL, mod[5], X,
+                         w.L, stream)
+
+    rnd = r0
+    for _ in range(args.warmup):
+        run_round(rnd)
+        rnd += 1
+    torch.cuda.synchronize(dev)
+    rounds = args.steps
+    rev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(rounds)]
+    clocks = ClockSampler(local)
+    time.sleep(0.3)
+    barrier(dist, dev)
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    for i in range(rounds):
+        rev[i][0].record(stream)
+        run_round(rnd)
+        rev[i][1].record(stream)
+        rnd += 1
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    barrier(dist, dev)
+    clocks.stop()
+    status = wf.wf_sync_status(plan, stream)
+    if status != wf.WF_OK:
+        raise SystemExit("device status %d (%s)" % (status, wf.status_string(status)))
+    per_round = [a.elapsed_time(b) for a, b in rev]
+    ms_round = allreduce_max(dist, sum(per_round), dev) / rounds
+    flops_round = w.layers * block_flops(w, hidden, ffn, wf.wf_useful_flops(plan, r0))
+    clk = clocks.summary(t_wall0, t_wall1)
+    plan.destroy()
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+    peak_tf = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    value = aggregate_tflops(world, flops_round, ms_round)
+    srt = sorted(per_round)
+    return {
+        "metric": "DiT rounds of the wave model: useful TFLOP/s, rounds/s (= output chunks/s)",
+        "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": rounds,
+        "warmup": args.warmup, "ms_per_step": round(ms_round, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded bf16 N(0,1) residual stream; random-init weights per layer)",
+        "config": {"workload": w.name, "layers": w.layers, "hidden": hidden, "ffn": ffn,
+                   "heads": w.H, "head_dim": w.D, "chunk_tokens": w.L, "wave_chunks": w.n_wave,
+                   "history_chunks": w.n_hist,
+                   "step": "one full round: %d DiT blocks (LN, QKV + norm/RoPE/append, attention, "
+                           "out-proj + gated residual, LN, FFN1 + GELU, FFN2 + gated residual)"
+                           % w.layers,
+                   "parallelism": "replica%d" % world,
+                   "l2": "no flush: per-layer rings and weights total %.1f GB" % (
+                       w.layers * (2 * w.R * w.L * w.H * w.D * 2 +
+                                   2 * (4 * hidden * w.H * w.D + 2 * hidden * ffn)) / 1e9)},
+        "round_ms_median": round(statistics.median(per_round), 3),
+        "round_ms_p90": round(srt[min(len(srt) - 1, int(0.9 * len(srt)))], 3),
+        "rounds_per_s": round(world * 1000.0 / ms_round, 3),
+        "latent_frames_per_s": round(world * 1000.0 / ms_round * w.F, 3),
+        "frac_sustained": round(value / world / peak_tf, 4),
+        "gpu_launches": 7 * w.layers * rounds,    # plus one torch copy of x0 per round
+        "clocks": clk,
+    }
+
+
 def run_round_loop(args, rank, world, local):
     """Full rounds of a multi-layer workload: every round runs, layer after layer,
     the append and the attention of each layer on that layer's own ring, then
@@ -954,6 +1068,8 @@ def main():
                     help="skip the DiT-block leg (timed after the attention step)")
     ap.add_argument("--attn", default="bf16", choices=["bf16", "fp8qk"],
                     help="attention variant: bf16 (default) or E4M3 Q.K^T with bf16 P.V")
+    ap.add_argument("--blocks", action="store_true",
+                    help="with a multi-layer workload: every layer runs the whole DiT block")
     ap.add_argument("--wp", type=int, default=0,
                     help="Wave Parallelism: under torchrun, split the wave over the ranks; "
                          "in one process, emulate N ranks on the one GPU (projected time)")
@@ -969,6 +1085,8 @@ def main():
         line = run_reference(args, rank, world)
     elif args.wp:
         line = run_wp(args, rank, world, local)
+    elif wi.WORKLOADS[args.workload].layers > 1 and args.blocks:
+        line = run_block_round_loop(args, rank, world, local)
     elif wi.WORKLOADS[args.workload].layers > 1:
         line = run_round_loop(args, rank, world, local)
     else:

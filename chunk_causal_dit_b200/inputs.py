@@ -172,6 +172,29 @@ def block_inputs(w: Workload, hidden: int, ffn: int, seed: int = 0) -> BlockInpu
         gamma_q=gq, gamma_k=gk)
 
 
+def block_weights_on(device, w: Workload, hidden: int, ffn: int, seed: int, layer: int):
+    """Random-init weights of one block drawn on `device` from a seeded generator
+    there (faster than host draws for many layers): the same recipe as
+    ``block_inputs`` (weights N(0, 1/in) in bf16, biases 0.02 N(0,1), modulation
+    0.1 N(0,1) per wave chunk), a different stream of numbers."""
+    g = torch.Generator(device=device)
+    g.manual_seed((int(seed) * 1009 + int(layer)) * 16 + STREAM_W)
+    HD = w.H * w.D
+
+    def wt(o, i):
+        return (torch.randn((o, i), generator=g, device=device) * i ** -0.5).to(torch.bfloat16)
+
+    def vec(shape, scale):
+        return torch.randn(shape, generator=g, device=device) * scale
+    return dict(w_qkv=wt(3 * HD, hidden), b_qkv=vec((3 * HD,), 0.02),
+                w_o=wt(hidden, HD), b_o=vec((hidden,), 0.02),
+                w_1=wt(ffn, hidden), b_1=vec((ffn,), 0.02),
+                w_2=wt(hidden, ffn), b_2=vec((hidden,), 0.02),
+                mod=vec((6, w.n_wave, hidden), 0.1),
+                gamma_q=(1.0 + 0.1 * torch.randn((w.H, w.D), generator=g, device=device)),
+                gamma_k=(1.0 + 0.1 * torch.randn((w.H, w.D), generator=g, device=device)))
+
+
 def bits(t: torch.Tensor) -> np.ndarray:
     """bf16 tensor -> numpy uint16 bit patterns (same memory order)."""
     return t.contiguous().view(torch.int16).numpy().view(np.uint16)
