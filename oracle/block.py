@@ -142,3 +142,32 @@ def qkv_project_append(x_bits, w_bits, bias, pos, gamma_q, gamma_k, H, D,
     if want_f64:
         return out + (q, k, v)
     return out
+
+
+def block_forward(x_bits, wts, mod, pos, cache, round_, n_wave, n_hist, H, D, L,
+                  eps=DEFAULT_EPS, split=None, theta=DEFAULT_THETA):
+    """One DiT block over a wave (reading s16 of the block's layers), composed from
+    the functions above; every intermediate the GPU stores is rounded once to bf16.
+
+    x_bits [T, C]; wts: dict of bf16 bits w_qkv, w_o, w_1, w_2 and fp32 b_qkv, b_o,
+    b_1, b_2, gamma_q, gamma_k; mod [6, n_wave, C] fp32 (shift, scale, gate of the
+    attention half, then of the feed-forward half; chunk c's tokens take row c);
+    pos [T, 3]; cache: an ``oracle.OracleCache`` holding the visible history
+    chunks (the wave's K/V are added here, under their absolute ids).
+    Returns the block's output x2 (bf16 bits [T, C]) and the intermediates.
+    """
+    from . import round_attention
+    T, C = x_bits.shape
+    h = layer_norm_modulate(x_bits, mod[0], mod[1], L)
+    q, k, v = qkv_project_append(h, wts["w_qkv"], wts["b_qkv"], pos, wts["gamma_q"],
+                                 wts["gamma_k"], H, D, eps, split, theta)
+    cache.put_wave(round_, k, v)
+    rows = np.repeat(np.arange(T), H)
+    heads = np.tile(np.arange(H), T)
+    o64, _ = round_attention(cache, round_, n_wave, n_hist, q, rows, heads)
+    o = f64_to_bf16(o64).reshape(T, H * D)
+    x1 = linear(o, wts["w_o"], wts["b_o"], "gated_residual", mod[2], x_bits, L)
+    h2 = layer_norm_modulate(x1, mod[3], mod[4], L)
+    f = linear(h2, wts["w_1"], wts["b_1"], "gelu_tanh")
+    x2 = linear(f, wts["w_2"], wts["b_2"], "gated_residual", mod[5], x1, L)
+    return x2, dict(h=h, q=q, k=k, v=v, o=o, x1=x1, h2=h2, f=f)

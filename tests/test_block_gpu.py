@@ -278,3 +278,72 @@ def test_full_size_sampled(wf):
     S = _abs_sum(h[rows], b.w_2) * np.abs(gate.numpy().astype(np.float64))[c_of]
     _assert_gemm_close(_bits(out)[rows], ref2, S, "ffn2 full size")
     plan.destroy()
+
+
+def test_block_composition(wf):
+    """The seven calls of one DiT block, composed as bench.py's block leg composes
+    them (gated residuals in place on the residual stream, ring with history),
+    against oracle.block.block_forward.  Bar: the two stored roundings of the
+    residual stream (x1 and x2) may each land one bf16 quantum apart from the
+    oracle's, and the attention's error (1e-2 max, 1e-3 mean on unit-scale data)
+    reaches x2 through W_o (unit gain) times a gate of ~0.1, so
+    |got - ref| <= 2 quanta(ref) + 1e-2 per element and mean |got - ref| <= 1e-3."""
+    import oracle
+    import oracle.block as ob
+    dev = "cuda"
+    F, gh, gw, W, Hh, H, D, ffn, r = 2, 6, 25, 3, 1, 2, 128, 512, 2
+    L, T, C, R = F * gh * gw, W * F * gh * gw, H * D, W + Hh
+    s = 21
+    x = wi.bf16_normal((T, C), s, wi.STREAM_X)
+    wts = dict(w_qkv=wi.bf16_weight(3 * C, C, s, 1), w_o=wi.bf16_weight(C, C, s, 2),
+               w_1=wi.bf16_weight(ffn, C, s, 3), w_2=wi.bf16_weight(C, ffn, s, 4),
+               b_qkv=wi.f32_vector((3 * C,), 0.02, s, wi.STREAM_BIAS, 1),
+               b_o=wi.f32_vector((C,), 0.02, s, wi.STREAM_BIAS, 2),
+               b_1=wi.f32_vector((ffn,), 0.02, s, wi.STREAM_BIAS, 3),
+               b_2=wi.f32_vector((C,), 0.02, s, wi.STREAM_BIAS, 4))
+    wts["gamma_q"], wts["gamma_k"] = wi.gains(H, D, s)
+    mod = wi.f32_vector((6, W, C), 0.1, s, wi.STREAM_MOD)
+    hk = wi.bf16_normal((Hh, L, H, D), s, 3)
+    hv = wi.bf16_normal((Hh, L, H, D), s, 4)
+    d = {k: t.to(dev) for k, t in wts.items()}
+    md = mod.to(dev)
+    plan = wf.Plan(L, W, Hh, H, D).set_rope(F, gh, gw)
+    kc = torch.zeros((R, L, H, D), dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros_like(kc)
+    for j in range(Hh):
+        kc[(r - Hh + j) % R].copy_(hk[j])
+        vc[(r - Hh + j) % R].copy_(hv[j])
+    X = x.to(dev)
+    h = torch.empty_like(X)
+    q_out = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+    o = torch.empty_like(q_out)
+    f = torch.empty((T, ffn), dtype=torch.bfloat16, device=dev)
+    wf.wf_layer_norm_modulate(plan, X, md[0], md[1], L, h)
+    wf.wf_qkv_proj_norm_rope_append(plan, r, h, d["w_qkv"], d["b_qkv"], d["gamma_q"],
+                                    d["gamma_k"], q_out, kc, vc)
+    wf.wf_chunk_causal_attn(plan, r, q_out, kc, vc, o)
+    wf.wf_linear(plan, o.view(T, C), d["w_o"], X, d["b_o"], wf.WF_EPI_GATED_RESIDUAL, md[2], X, L)
+    wf.wf_layer_norm_modulate(plan, X, md[3], md[4], L, h)
+    wf.wf_linear(plan, h, d["w_1"], f, d["b_1"], wf.WF_EPI_GELU_TANH)
+    wf.wf_linear(plan, f, d["w_2"], X, d["b_2"], wf.WF_EPI_GATED_RESIDUAL, md[5], X, L)
+    torch.cuda.synchronize()
+    assert wf.wf_sync_status(plan) == wf.WF_OK
+    cache = oracle.OracleCache(L)
+    for j in range(Hh):
+        cache.put(r - Hh + j, _bits(hk[j]), _bits(hv[j]))
+    bw = {k: (_bits(t) if t.dtype == torch.bfloat16 else t.numpy()) for k, t in wts.items()}
+    x2, inter = ob.block_forward(_bits(x), bw, mod.numpy(), oracle.positions(r, W, F, gh, gw),
+                                 cache, r, W, Hh, H, D, L)
+    ref = oracle.bf16_to_f64(x2)
+    got = _f64(X.float())
+    diff = np.abs(got - ref)
+    tol = 2.0 * bf16_quantum(ref) + 1e-2
+    assert not (diff > tol).any(), "block: %d outside the bar (max %g)" % (
+        int((diff > tol).sum()), float(diff.max()))
+    assert diff.mean() <= 1e-3, "block: mean abs %g" % diff.mean()
+    # the ring holds the wave's K/V where the attention read them
+    for c in range(W):
+        got_k = _bits(kc[(r + c) % R])
+        want_k = inter["k"][c * L:(c + 1) * L]
+        assert (got_k != want_k).mean() < 0.05        # bf16 roundings of the fused epilogue
+    plan.destroy()

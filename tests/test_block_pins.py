@@ -11,7 +11,9 @@ Each pin ties the oracle to something other than itself:
   so the output is the shift itself), per-chunk modulation rows;
 * QKV projection with the fused norm/RoPE/append: with W = [I; I; I] it must
   reduce bit for bit to the (separately pinned) append oracle applied to x, and
-  permuting W's heads permutes the outputs' heads.
+  permuting W's heads permutes the outputs' heads;
+* the composed block: zero gates return the input bit for bit, and with the
+  feed-forward gate zero the block is the gated attention half of its parts.
 """
 import math
 
@@ -133,3 +135,53 @@ def test_qkv_head_permutation():
     pq, pk, pv = ob.qkv_project_append(x, w[rows], bias[rows], pos, gq[perm], gk[perm], H, D)
     assert np.array_equal(pq, q[:, perm]) and np.array_equal(pk, k[:, perm])
     assert np.array_equal(pv, v[:, perm])
+
+
+def _block_case(seed, F=1, gh=2, gw=8, W=2, Hh=1, H=2, D=64, ffn=96, r=1):
+    g = np.random.default_rng(seed)
+    L = F * gh * gw
+    T, C = W * L, H * D
+    wts = dict(w_qkv=_rand_bits(g, (3 * C, C), 0.1), w_o=_rand_bits(g, (C, C), 0.1),
+               w_1=_rand_bits(g, (ffn, C), 0.1), w_2=_rand_bits(g, (C, ffn), 0.1),
+               b_qkv=g.standard_normal(3 * C).astype(np.float32) * 0.02,
+               b_o=g.standard_normal(C).astype(np.float32) * 0.02,
+               b_1=g.standard_normal(ffn).astype(np.float32) * 0.02,
+               b_2=g.standard_normal(C).astype(np.float32) * 0.02,
+               gamma_q=(1 + 0.1 * g.standard_normal((H, D))).astype(np.float32),
+               gamma_k=(1 + 0.1 * g.standard_normal((H, D))).astype(np.float32))
+    mod = (0.1 * g.standard_normal((6, W, C))).astype(np.float32)
+    x = _rand_bits(g, (T, C))
+    cache = oracle.OracleCache(L)
+    for j in range(min(Hh, r)):
+        cache.put(r - 1 - j, _rand_bits(g, (L, H, D)), _rand_bits(g, (L, H, D)))
+    pos = oracle.positions(r, W, F, gh, gw)
+    return x, wts, mod, pos, cache, dict(round_=r, n_wave=W, n_hist=Hh, H=H, D=D, L=L)
+
+
+def test_block_forward_zero_gates_return_the_input():
+    x, wts, mod, pos, cache, kw = _block_case(11)
+    mod[2] = 0.0
+    mod[5] = 0.0
+    x2, inter = ob.block_forward(x, wts, mod, pos, cache, **kw)
+    assert np.array_equal(x2, x) and np.array_equal(inter["x1"], x)
+
+
+def test_block_forward_attention_half_matches_its_parts():
+    """With the feed-forward gate zero, the block is x + gate * (o W_o^T + b_o) of
+    the chunk-causal attention over the fused projection's q/k/v (the parts
+    pinned separately), and the ring holds the wave's K/V under their ids."""
+    x, wts, mod, pos, cache, kw = _block_case(12)
+    mod[5] = 0.0
+    x2, inter = ob.block_forward(x, wts, mod, pos, cache, **kw)
+    L, H, D, W, r = kw["L"], kw["H"], kw["D"], kw["n_wave"], kw["round_"]
+    h = ob.layer_norm_modulate(x, mod[0], mod[1], L)
+    q, k, v = ob.qkv_project_append(h, wts["w_qkv"], wts["b_qkv"], pos, wts["gamma_q"],
+                                    wts["gamma_k"], H, D)
+    for c in range(W):
+        assert np.array_equal(cache.chunks[r + c][0], k[c * L:(c + 1) * L])
+    T = W * L
+    rows, heads = np.repeat(np.arange(T), H), np.tile(np.arange(H), T)
+    o64, _ = oracle.round_attention(cache, r, W, kw["n_hist"], q, rows, heads)
+    o = oracle.f64_to_bf16(o64).reshape(T, H * D)
+    want = ob.linear(o, wts["w_o"], wts["b_o"], "gated_residual", mod[2], x, L)
+    assert np.array_equal(x2, want)
