@@ -51,17 +51,20 @@ constexpr uint32_t kABytes = BM * BK * 2;              // 16 KB
 constexpr uint32_t kBBytes = (BN / 2) * BK * 2;        // 16 KB: this CTA's 128 rows of B
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
 constexpr int kTabMax = 3072;                          // float2 entries (24 KB)
+constexpr uint32_t kStageRowBytes = 80;                // epilogue staging (see warp_store32)
+constexpr uint32_t kWarpStageBytes = 32 * kStageRowBytes;
 constexpr uint32_t kTmemCols = 512;
 constexpr unsigned long long kDrainLimit = 1ull << 32;
 
 // Shared-memory plan per epilogue: the stage ring, then (QKV only) the RoPE
-// (cos, sin) tables, then the barrier block.  (A seventh stage fits without the
-// tables; measured on B200 it was 1-4% slower than six.)
+// (cos, sin) tables, the epilogue warps' staging buffers and the barrier block.
+// (Six stages measured 1-4% faster than seven; with the tables only five fit.)
 template <int Epi>
 struct Smem {
-    static constexpr int kStages = 6;
+    static constexpr int kStages = Epi == kEpiQkvAppend ? 5 : 6;
     static constexpr uint32_t kTabOff = kStages * kStageBytes;
-    static constexpr uint32_t kBarOff = kTabOff + (Epi == kEpiQkvAppend ? kTabMax * 8 : 0);
+    static constexpr uint32_t kStgOff = kTabOff + (Epi == kEpiQkvAppend ? kTabMax * 8 : 0);
+    static constexpr uint32_t kBarOff = kStgOff + kEpiWarps * kWarpStageBytes;
     static constexpr uint32_t kBytes = kBarOff + 256 + 1024;   // + 1024-byte alignment slack
     // barrier indices
     static constexpr int full = 0, empty = kStages, acc_full = 2 * kStages,
@@ -135,10 +138,60 @@ __device__ __forceinline__ void unpack8(const uint4 &u, float *x)
     }
 }
 
+// Each epilogue warp moves its 32 rows x 32 columns of bf16 through a staging
+// buffer of its own in shared memory, so that global loads and stores are
+// coalesced: 8 rows x 64 contiguous bytes per instruction instead of one
+// 16-byte piece of each of 32 rows (measured: that pattern cost the K = 1536
+// projections ~14% of their time).  Rows are 80 bytes apart (64 + 16 of
+// padding), which makes the 16-byte shared stores of a warp conflict-free.
+
+// Store: thread `lane` holds its row's 32 values packed in w; dst is that row's
+// destination (nullptr: the row stores nothing).  Warp-collective.
+__device__ __forceinline__ void warp_store32(uint8_t *stage, const uint4 (&w)[4], uint16_t *dst)
+{
+    const int lane = threadIdx.x & 31;
+    uint4 *mine = reinterpret_cast<uint4 *>(stage + lane * kStageRowBytes);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) mine[j] = w[j];
+    __syncwarp();
+    const unsigned long long d = reinterpret_cast<unsigned long long>(dst);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int piece = 32 * i + lane, rr = piece >> 2, part = piece & 3;
+        const unsigned long long drow = __shfl_sync(0xFFFFFFFFu, d, rr);
+        const uint4 v = *reinterpret_cast<const uint4 *>(stage + rr * kStageRowBytes + part * 16);
+        if (drow != 0ull) reinterpret_cast<uint4 *>(drow)[part] = v;
+    }
+    __syncwarp();
+}
+
+// Load: src is this thread's row (nullptr: zeros); w receives the row's 32 values.
+// Warp-collective.
+__device__ __forceinline__ void warp_load32(uint8_t *stage, const uint16_t *src, uint4 (&w)[4])
+{
+    const int lane = threadIdx.x & 31;
+    const unsigned long long s = reinterpret_cast<unsigned long long>(src);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int piece = 32 * i + lane, rr = piece >> 2, part = piece & 3;
+        const unsigned long long srow = __shfl_sync(0xFFFFFFFFu, s, rr);
+        *reinterpret_cast<uint4 *>(stage + rr * kStageRowBytes + part * 16) =
+            srow != 0ull ? __ldg(reinterpret_cast<const uint4 *>(srow) + part)
+                         : make_uint4(0u, 0u, 0u, 0u);
+    }
+    __syncwarp();
+    const uint4 *mine = reinterpret_cast<const uint4 *>(stage + lane * kStageRowBytes);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) w[j] = mine[j];
+    __syncwarp();
+}
+
 // 32 columns [c, c + 32) of one row: bias, activation / gated residual, bf16 store.
+// Warp-collective (row_ok false: the row takes part but loads and stores nothing).
 template <int Epi>
 __device__ __forceinline__ void finish32(const GemmParams &p, const uint32_t (&r)[32], long row,
-                                         int c, const float *gate_row)
+                                         bool row_ok, int c, const float *gate_row,
+                                         uint8_t *stage)
 {
     float v[32];
 #pragma unroll
@@ -159,26 +212,29 @@ __device__ __forceinline__ void finish32(const GemmParams &p, const uint32_t (&r
         for (int i = 0; i < 32; ++i) v[i] = gelu_tanh(v[i]);
     }
     if constexpr (Epi == kEpiGatedResidual) {
-        const uint4 *r4 = reinterpret_cast<const uint4 *>(p.resid + row * p.N + c);
+        uint4 rw[4];
+        warp_load32(stage, row_ok ? p.resid + row * p.N + c : nullptr, rw);
         const float4 *g4 = reinterpret_cast<const float4 *>(gate_row + c);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             float x[8];
-            unpack8(__ldg(r4 + j), x);
+            unpack8(rw[j], x);
             const float4 ga = __ldg(g4 + 2 * j), gb = __ldg(g4 + 2 * j + 1);
             const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
 #pragma unroll
             for (int e = 0; e < 8; ++e) v[8 * j + e] = fmaf(g[e], v[8 * j + e], x[e]);
         }
     }
-    uint4 *dst = reinterpret_cast<uint4 *>(p.c + row * p.N + c);
+    uint4 w[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) dst[j] = pack8(v + 8 * j);
+    for (int j = 0; j < 4; ++j) w[j] = pack8(v + 8 * j);
+    warp_store32(stage, w, row_ok ? p.c + row * p.N + c : nullptr);
 }
 
 // Linear epilogues: this thread's row, 128 columns from col0 (TMEM at taddr).
 template <int Epi>
-__device__ __forceinline__ void epi_linear(const GemmParams &p, uint32_t taddr, long row, int col0)
+__device__ __forceinline__ void epi_linear(const GemmParams &p, uint32_t taddr, long row, int col0,
+                                           uint8_t *stage)
 {
     const bool row_ok = row < p.M;
     const float *gate_row = nullptr;
@@ -190,10 +246,9 @@ __device__ __forceinline__ void epi_linear(const GemmParams &p, uint32_t taddr, 
         tmem_ld32(taddr + 64 * h, r0);
         tmem_ld32(taddr + 64 * h + 32, r1);
         tmem_wait_ld();
-        const int c = col0 + 64 * h;
-        if (!row_ok) continue;
-        if (c < p.N) finish32<Epi>(p, r0, row, c, gate_row);
-        if (c + 32 < p.N) finish32<Epi>(p, r1, row, c + 32, gate_row);
+        const int c = col0 + 64 * h;                 // warp-uniform column guards
+        if (c < p.N) finish32<Epi>(p, r0, row, row_ok, c, gate_row, stage);
+        if (c + 32 < p.N) finish32<Epi>(p, r1, row, row_ok, c + 32, gate_row, stage);
     }
 }
 
@@ -207,7 +262,7 @@ __device__ __forceinline__ void epi_linear(const GemmParams &p, uint32_t taddr, 
 // squares first), with the next chunk's load in flight while one is processed.
 template <int D>
 __device__ __forceinline__ void epi_qkv(const GemmParams &p, uint32_t taddr, long row, int col0,
-                                        const float2 *tab)
+                                        const float2 *tab, uint8_t *stage)
 {
     constexpr int kHeads = 128 / D;
     constexpr int kChunks = D / 32;
@@ -275,7 +330,7 @@ __device__ __forceinline__ void epi_qkv(const GemmParams &p, uint32_t taddr, lon
 #pragma unroll
         for (int j = 0; j < kChunks; ++j) {
             if (j + 1 < kChunks) tmem_ld32(ta + 32 * (j + 1), r[(j + 1) & 1]);
-            if (ok) {
+            {
                 float v[32];
 #pragma unroll
                 for (int q4 = 0; q4 < 8; ++q4) {
@@ -302,9 +357,10 @@ __device__ __forceinline__ void epi_qkv(const GemmParams &p, uint32_t taddr, lon
                         }
                     }
                 }
-                uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * j);
+                uint4 w[4];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) d4[q] = pack8(v + 8 * q);
+                for (int q = 0; q < 4; ++q) w[q] = pack8(v + 8 * q);
+                warp_store32(stage, w, ok ? dst + 32 * j : nullptr);
             }
             tmem_wait_ld();
         }
@@ -467,6 +523,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
         const int lq = warp & 3;                   // TMEM lane quarter of this warp
         const int half = (warp - 2) >> 2;          // 128-column half of the tile
         const float2 *tab = reinterpret_cast<const float2 *>(smem + B::kTabOff);
+        uint8_t *stage = smem + B::kStgOff + (warp - 2) * kWarpStageBytes;
         uint32_t acc_it = 0;
         for (int t = cid; t < p.n_tiles; t += ncl, ++acc_it) {
             const uint32_t b = acc_it & 1u;
@@ -480,9 +537,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
             const uint32_t taddr =
                 tmem + (static_cast<uint32_t>(lq * 32) << 16) + b * BN + half * (BN / 2);
             if constexpr (Epi == kEpiQkvAppend)
-                epi_qkv<D>(p, taddr, row, col0, tab);
+                epi_qkv<D>(p, taddr, row, col0, tab, stage);
             else
-                epi_linear<Epi>(p, taddr, row, col0);
+                epi_linear<Epi>(p, taddr, row, col0, stage);
             // the accumulator may be overwritten once this warp's TMEM loads are done
             // (tcgen05.wait::ld above): a relaxed arrive, so that the epilogue's global
             // stores need not drain first, as a release at cluster scope would demand
