@@ -1,6 +1,11 @@
 """Build libwf.so in-tree with nvcc for sm_100a (B200).
 
-    python -m chunk_causal_dit_b200.build [--force] [--verbose]
+    python -m chunk_causal_dit_b200.build [--force] [--verbose] [--check]
+
+--check builds the debug variant libwf_check.so (compiled with -DWF_CHECK: the
+kernels' computed global indices are bounds-checked, a failure is reported by
+wf_sync_status as WF_ERR_BOUNDS instead of trapping).  The binding loads it
+instead of libwf.so when WF_LIB_VARIANT=check is set in the environment.
 
 The library is written next to this file (chunk_causal_dit_b200/libwf.so) so
 that it travels with the source tree; the CUDA runtime is linked statically,
@@ -19,9 +24,10 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libwf.so")
+LIB_CHECK = os.path.join(HERE, "libwf_check.so")
 SOURCES = ["wf_api.cu", "append_kernel.cu", "attn_kernel.cu", "attn_pair_kernel.cu",
            "quant_fp8_kernel.cu", "noalloc.cu", "gemm_kernel.cu", "ln_kernel.cu"]
-HEADERS = ["sm100.cuh", "wf_internal.h", "exp2_poly.h"]
+HEADERS = ["sm100.cuh", "wf_internal.h", "exp2_poly.h", "wf_check.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -38,34 +44,36 @@ def _inputs():
     return files
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(f) <= t for f in _inputs())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
+def build(force: bool = False, verbose: bool = False, check: bool = False) -> str:
+    lib = LIB_CHECK if check else LIB
+    if not force and up_to_date(lib):
+        return lib
     nvcc = os.environ.get("NVCC", "nvcc")
-    tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = [nvcc, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp,
-           *[os.path.join(CSRC, s) for s in SOURCES]]
+    tmp = lib + ".tmp%d" % os.getpid()
+    cmd = [nvcc, *NVCC_FLAGS, *(["-DWF_CHECK"] if check else []), "-I", INCLUDE, "-I", CSRC,
+           "-o", tmp, *[os.path.join(CSRC, s) for s in SOURCES]]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
+    ap.add_argument("--check", action="store_true", help="build the WF_CHECK debug variant")
     a = ap.parse_args(argv)
-    print(build(force=a.force, verbose=a.verbose))
+    print(build(force=a.force, verbose=a.verbose, check=a.check))
 
 
 if __name__ == "__main__":

@@ -19,6 +19,7 @@
 #include <cuda_bf16.h>
 
 #include "sm100.cuh"
+#include "wf_check.cuh"
 #include "wf_internal.h"
 
 namespace wf {
@@ -49,7 +50,8 @@ __device__ __forceinline__ uint4 pack8(const float (&y)[8])
 }
 
 template <int D>
-__global__ void __launch_bounds__(kMaxThreads) qk_norm_rope_append_kernel(const AppendParams p)
+__global__ void __launch_bounds__(kMaxThreads) qk_norm_rope_append_kernel(const AppendParams p,
+                                                                          DeviceWords *words)
 {
     constexpr int TPR = D / 8;           // threads per (token, head) row
     constexpr int NP = D / 2;            // RoPE pairs
@@ -118,7 +120,9 @@ __global__ void __launch_bounds__(kMaxThreads) qk_norm_rope_append_kernel(const 
         s_cs[tl][pr] = make_float2(cs, sn);
         if (pr == 0) {
             const int slot = ring_slot(p.round + c, p.R);
-            s_off[tl] = (static_cast<long>(slot) * p.L + ic) * p.H * D;
+            const bool in = WF_BOUNDS(slot >= 0 && slot < p.R && c < p.W && ic < p.L, words,
+                                      kSiteAppend);
+            s_off[tl] = in ? (static_cast<long>(slot) * p.L + ic) * p.H * D : -1;
         }
     }
     __syncthreads();
@@ -154,7 +158,7 @@ __global__ void __launch_bounds__(kMaxThreads) qk_norm_rope_append_kernel(const 
             yk[2 * e] = k0 * cs.x - k1 * cs.y;
             yk[2 * e + 1] = k0 * cs.y + k1 * cs.x;
         }
-        if (active) {
+        if (active && WF_CHECKED(s_off[tl] >= 0)) {
             const long off = (n * p.H + h) * D + part * 8;
             const long coff = s_off[tl] + static_cast<long>(h) * D + part * 8;
             *reinterpret_cast<uint4 *>(p.q_out + off) = pack8(yq);
@@ -166,7 +170,7 @@ __global__ void __launch_bounds__(kMaxThreads) qk_norm_rope_append_kernel(const 
 
 }  // namespace
 
-cudaError_t launch_append(const AppendParams &p_in, int D, cudaStream_t stream)
+cudaError_t launch_append(const AppendParams &p_in, int D, cudaStream_t stream, DeviceWords *words)
 {
     AppendParams p = p_in;
     const int tpr = D / 8;
@@ -179,9 +183,9 @@ cudaError_t launch_append(const AppendParams &p_in, int D, cudaStream_t stream)
     if (bx <= 0) return cudaSuccess;
     const dim3 grid(static_cast<unsigned>(bx), static_cast<unsigned>(by));
     if (D == 128)
-        qk_norm_rope_append_kernel<128><<<grid, threads, 0, stream>>>(p);
+        qk_norm_rope_append_kernel<128><<<grid, threads, 0, stream>>>(p, words);
     else
-        qk_norm_rope_append_kernel<64><<<grid, threads, 0, stream>>>(p);
+        qk_norm_rope_append_kernel<64><<<grid, threads, 0, stream>>>(p, words);
     return cudaGetLastError();
 }
 

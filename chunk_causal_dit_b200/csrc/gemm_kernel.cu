@@ -36,6 +36,7 @@
 #include <atomic>
 
 #include "sm100.cuh"
+#include "wf_check.cuh"
 #include "wf_internal.h"
 
 namespace wf {
@@ -228,7 +229,8 @@ __device__ __forceinline__ void finish32(const GemmParams &p, const uint32_t (&r
     uint4 w[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) w[j] = pack8(v + 8 * j);
-    warp_store32(stage, w, row_ok ? p.c + row * p.N + c : nullptr);
+    const bool st = row_ok && WF_BOUNDS(c + 32 <= p.N, p.words, kSiteGemmStore);
+    warp_store32(stage, w, st ? p.c + row * p.N + c : nullptr);
 }
 
 // Linear epilogues: this thread's row, 128 columns from col0 (TMEM at taddr).
@@ -267,12 +269,14 @@ __device__ __forceinline__ void epi_qkv(const GemmParams &p, uint32_t taddr, lon
     constexpr int kHeads = 128 / D;
     constexpr int kChunks = D / 32;
     const int HD = p.H * D;
-    const bool ok = row < p.M && col0 < p.N;
     const int which = col0 / HD;                 // 0 q, 1 k, 2 v (warp-uniform)
     const int h0 = (col0 - which * HD) / D;
-    const long n = ok ? row : 0;                 // rows past M store nothing
+    const long n = row < p.M ? row : 0;          // rows past M store nothing
     const int c = static_cast<int>(n / p.L);
     const int ic = static_cast<int>(n - static_cast<long>(c) * p.L);
+    const bool ok = row < p.M && col0 < p.N &&
+                    WF_BOUNDS(which <= 2 && h0 + kHeads <= p.H && c < p.W && ic < p.L, p.words,
+                              kSiteGemmQkv);
     const int hw = p.rope.gh * p.rope.gw;
     const int f = ic / hw;
     const int rem = ic - f * hw;
@@ -350,8 +354,10 @@ __device__ __forceinline__ void epi_qkv(const GemmParams &p, uint32_t taddr, lon
                             const int pr = 16 * j + pl;          // pair within the head
                             const float a = v[2 * pl] * rs * (e ? g.z : g.x);
                             const float bb = v[2 * pl + 1] * rs * (e ? g.w : g.y);
+                            const int ti = pr < nt ? it + pr : (pr < nt + nh ? ih + pr : iw + pr);
                             const float2 cs =
-                                tab[pr < nt ? it + pr : (pr < nt + nh ? ih + pr : iw + pr)];
+                                WF_BOUNDS(ti >= 0 && ti < p.n_tab, p.words, kSiteGemmTable)
+                                    ? tab[ti] : make_float2(1.0f, 0.0f);
                             v[2 * pl] = a * cs.x - bb * cs.y;
                             v[2 * pl + 1] = a * cs.y + bb * cs.x;
                         }

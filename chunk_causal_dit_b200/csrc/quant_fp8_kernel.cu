@@ -16,6 +16,7 @@
 // Both kernels are HBM-bound: 2 bytes read and 1 byte written per element.
 #include <cuda_bf16.h>
 
+#include "wf_check.cuh"
 #include "wf_internal.h"
 
 namespace wf {
@@ -66,7 +67,7 @@ template <int D>
 __global__ void __launch_bounds__(256) quantize_rows_kernel(const uint16_t *__restrict__ q,
                                                             uint8_t *__restrict__ q8,
                                                             float *__restrict__ scale, long n_rows,
-                                                            int H)
+                                                            int H, DeviceWords *words)
 {
     constexpr int kLanesPerRow = D / 8;
     constexpr int kRowsPerLoad = 32 / kLanesPerRow;
@@ -108,7 +109,8 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const uint16_t *__re
             if (part == 0) {
                 const long n = row / H;
                 const int h = static_cast<int>(row - n * H);
-                scale[static_cast<long>(h) * n_tok + n] = fp8_scale(a);
+                if (WF_BOUNDS(n < n_tok && h < H, words, kSiteQuantRows))
+                    scale[static_cast<long>(h) * n_tok + n] = fp8_scale(a);
             }
         }
     }
@@ -123,7 +125,8 @@ template <int D>
 __global__ void __launch_bounds__(256) quantize_tiles_kernel(const uint16_t *__restrict__ k,
                                                              uint8_t *__restrict__ k8,
                                                              float *__restrict__ scale,
-                                                             long first_chunk, int L, int H, int R)
+                                                             long first_chunk, int L, int H, int R,
+                                                             DeviceWords *words)
 {
     constexpr int kLanesPerRow = D / 8;
     constexpr int kRowsPerLoad = 32 / kLanesPerRow;
@@ -134,6 +137,8 @@ __global__ void __launch_bounds__(256) quantize_tiles_kernel(const uint16_t *__r
     const int t = blockIdx.x - chunk * n_tiles;
     const int h = blockIdx.y;
     const int slot = ring_slot(first_chunk + chunk, R);
+    if (!WF_BOUNDS(slot >= 0 && slot < R && t < n_tiles && h < H, words, kSiteQuantTiles))
+        return;                                  // whole block: uniform
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int sub = lane / kLanesPerRow, part = lane % kLanesPerRow;
     const long slot_base = static_cast<long>(slot) * L;
@@ -177,28 +182,31 @@ __global__ void __launch_bounds__(256) quantize_tiles_kernel(const uint16_t *__r
 }  // namespace
 
 cudaError_t launch_quantize_rows(const uint16_t *q, uint8_t *q8, float *scale, long n_rows, int H,
-                                 int D, cudaStream_t stream)
+                                 int D, cudaStream_t stream, DeviceWords *words)
 {
     if (n_rows == 0) return cudaSuccess;
     const long rows_per_block = 8L * 4 * (32 / (D / 8));
     const dim3 grid(static_cast<unsigned>((n_rows + rows_per_block - 1) / rows_per_block));
     if (D == 128)
-        quantize_rows_kernel<128><<<grid, 256, 0, stream>>>(q, q8, scale, n_rows, H);
+        quantize_rows_kernel<128><<<grid, 256, 0, stream>>>(q, q8, scale, n_rows, H, words);
     else
-        quantize_rows_kernel<64><<<grid, 256, 0, stream>>>(q, q8, scale, n_rows, H);
+        quantize_rows_kernel<64><<<grid, 256, 0, stream>>>(q, q8, scale, n_rows, H, words);
     return cudaGetLastError();
 }
 
 cudaError_t launch_quantize_tiles(const uint16_t *k, uint8_t *k8, float *scale, long first_chunk,
-                                  int n_chunks, int L, int H, int R, int D, cudaStream_t stream)
+                                  int n_chunks, int L, int H, int R, int D, cudaStream_t stream,
+                                  DeviceWords *words)
 {
     if (n_chunks == 0) return cudaSuccess;
     const int n_tiles = (L + 127) / 128;
     const dim3 grid(static_cast<unsigned>(n_chunks * n_tiles), static_cast<unsigned>(H));
     if (D == 128)
-        quantize_tiles_kernel<128><<<grid, 256, 0, stream>>>(k, k8, scale, first_chunk, L, H, R);
+        quantize_tiles_kernel<128><<<grid, 256, 0, stream>>>(k, k8, scale, first_chunk, L, H, R,
+                                                               words);
     else
-        quantize_tiles_kernel<64><<<grid, 256, 0, stream>>>(k, k8, scale, first_chunk, L, H, R);
+        quantize_tiles_kernel<64><<<grid, 256, 0, stream>>>(k, k8, scale, first_chunk, L, H, R,
+                                                              words);
     return cudaGetLastError();
 }
 

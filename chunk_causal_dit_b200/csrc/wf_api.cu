@@ -9,10 +9,11 @@
 #include <new>
 
 #include "wf.h"
+#include "wf_check.cuh"
 #include "wf_internal.h"
 
 namespace wf {
-cudaError_t launch_append(const AppendParams &p, int D, cudaStream_t stream);
+cudaError_t launch_append(const AppendParams &p, int D, cudaStream_t stream, DeviceWords *words);
 cudaError_t launch_attn(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                         const AttnParams &p, int D, int grid, cudaStream_t stream);
 cudaError_t launch_attn_pair(const CUtensorMap &mq, const CUtensorMap &mk64, const CUtensorMap &mv,
@@ -20,9 +21,10 @@ cudaError_t launch_attn_pair(const CUtensorMap &mq, const CUtensorMap &mk64, con
 cudaError_t launch_attn_fp8qk(const CUtensorMap &mq8, const CUtensorMap &mk8, const CUtensorMap &mv,
                               const AttnParams &p, int grid, cudaStream_t stream);
 cudaError_t launch_quantize_rows(const uint16_t *q, uint8_t *q8, float *scale, long n_rows, int H,
-                                 int D, cudaStream_t stream);
+                                 int D, cudaStream_t stream, DeviceWords *words);
 cudaError_t launch_quantize_tiles(const uint16_t *k, uint8_t *k8, float *scale, long first_chunk,
-                                  int n_chunks, int L, int H, int R, int D, cudaStream_t stream);
+                                  int n_chunks, int L, int H, int R, int D, cudaStream_t stream,
+                                  DeviceWords *words);
 cudaError_t launch_gemm(const CUtensorMap &ma, const CUtensorMap &mb, const GemmParams &p, int epi,
                         cudaStream_t stream);
 int gemm_tab_max();
@@ -331,7 +333,7 @@ int wf_qk_norm_rope_append(wf_plan_t p, long round, const void *q, const void *k
     a.H = p->H;
     a.eps = static_cast<float>(p->eps);
     a.rope = p->rope;
-    cudaError_t e = wf::launch_append(a, p->D, static_cast<cudaStream_t>(stream));
+    cudaError_t e = wf::launch_append(a, p->D, static_cast<cudaStream_t>(stream), p->words);
     return e == cudaSuccess ? WF_OK : WF_ERR_CUDA;
 }
 
@@ -391,7 +393,7 @@ int wf_quantize_q_fp8(wf_plan_t p, const void *q_out, void *q8, float *q_scale, 
     const long rows = static_cast<long>(p->L) * p->W * p->H;
     cudaError_t e = wf::launch_quantize_rows(static_cast<const uint16_t *>(q_out),
                                              static_cast<uint8_t *>(q8), q_scale, rows, p->H, p->D,
-                                             static_cast<cudaStream_t>(stream));
+                                             static_cast<cudaStream_t>(stream), p->words);
     return e == cudaSuccess ? WF_OK : WF_ERR_CUDA;
 }
 
@@ -405,7 +407,7 @@ int wf_quantize_k_fp8(wf_plan_t p, long first_chunk, int n_chunks, const void *k
     cudaError_t e = wf::launch_quantize_tiles(static_cast<const uint16_t *>(k_cache),
                                               static_cast<uint8_t *>(k8_cache), k_scale, first_chunk,
                                               n_chunks, p->L, p->H, p->R, p->D,
-                                              static_cast<cudaStream_t>(stream));
+                                              static_cast<cudaStream_t>(stream), p->words);
     return e == cudaSuccess ? WF_OK : WF_ERR_CUDA;
 }
 
@@ -564,6 +566,7 @@ int wf_sync_status(wf_plan_t p, void *stream)
         cudaStreamSynchronize(st) != cudaSuccess)
         return WF_ERR_CUDA;
     if (host.status & wf::kStatusTimeout) return WF_ERR_TIMEOUT;
+    if (host.status & wf::kStatusBounds) return WF_ERR_BOUNDS;
     return WF_OK;
 }
 
@@ -594,6 +597,7 @@ const char *wf_status_string(int s)
     case WF_ERR_TIMEOUT: return "device wait timed out";
     case WF_ERR_NO_DEVICE: return "plan has no device state";
     case WF_ERR_DEVICE: return "device is not sm_100";
+    case WF_ERR_BOUNDS: return "bounds check failed (debug build)";
     default: return "unknown status";
     }
 }

@@ -11,7 +11,9 @@ import os
 from typing import Optional
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libwf.so")
+# WF_LIB_VARIANT=check selects the bounds-checked debug build (build.py --check)
+LIB_PATH = os.path.join(HERE, "libwf_check.so" if os.environ.get("WF_LIB_VARIANT") == "check"
+                        else "libwf.so")
 
 WF_OK = 0
 WF_ERR_INVALID_ARG = 1
@@ -20,6 +22,7 @@ WF_ERR_CUDA = 3
 WF_ERR_TIMEOUT = 4
 WF_ERR_NO_DEVICE = 5
 WF_ERR_DEVICE = 6
+WF_ERR_BOUNDS = 7
 
 # attention kernel variants (wf_plan_set_attn_kernel)
 WF_ATTN_AUTO = 0

@@ -59,7 +59,8 @@ typedef enum wf_status {
     WF_ERR_CUDA = 3,          /* a CUDA runtime/driver call or launch failed       */
     WF_ERR_TIMEOUT = 4,       /* a bounded device wait expired (kernel stopped)    */
     WF_ERR_NO_DEVICE = 5,     /* the plan has no device state (no GPU at wf_plan)  */
-    WF_ERR_DEVICE = 6         /* the device is not an sm_100 (B200-class) part     */
+    WF_ERR_DEVICE = 6,        /* the device is not an sm_100 (B200-class) part     */
+    WF_ERR_BOUNDS = 7         /* a bounds check of the WF_CHECK debug build failed */
 } wf_status;
 
 typedef struct wf_plan_s *wf_plan_t;
@@ -257,7 +258,9 @@ WF_API int wf_layer_norm_modulate(wf_plan_t plan, int M, int C, const void *x, c
                                   const float *scale, int rows_per_group, void *y, void *stream);
 
 /* Wait for `stream`, then read and clear the plan's device status word.
- * Returns WF_OK, WF_ERR_TIMEOUT (a bounded device wait expired) or WF_ERR_CUDA. */
+ * Returns WF_OK, WF_ERR_TIMEOUT (a bounded device wait expired), WF_ERR_BOUNDS
+ * (only in the debug build libwf_check.so, compiled with -DWF_CHECK: a computed
+ * index fell outside its tensor; the access was skipped) or WF_ERR_CUDA. */
 WF_API int wf_sync_status(wf_plan_t plan, void *stream);
 
 /* The key chunks the attention kernel visits in round r, in visiting order:

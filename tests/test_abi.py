@@ -225,3 +225,18 @@ def test_block_calls_validate_before_the_device(wf):
         assert ln(p.handle, 10, 64, f, f, f, 1, f, None) == N
     for q in (p, pg, p1, big, wide):
         q.destroy()
+
+
+def test_debug_build_exports_the_same_abi():
+    """libwf_check.so (the WF_CHECK variant) loads without a GPU, exports every
+    function the header declares, and names the status its checks report."""
+    import ctypes
+    import re
+    from chunk_causal_dit_b200 import build as wf_build
+    path = wf_build.build(check=True)
+    lib = ctypes.CDLL(path)
+    with open(os.path.join(ROOT, "include", "wf.h")) as f:
+        names = set(re.findall(r"WF_API\s+[^()]*?\b(wf_[a-z0-9_]+)\s*\(", f.read()))
+    assert names and all(hasattr(lib, n) for n in names)
+    lib.wf_status_string.restype = ctypes.c_char_p
+    assert b"bounds" in lib.wf_status_string(7)

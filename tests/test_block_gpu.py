@@ -347,3 +347,51 @@ def test_block_composition(wf):
         want_k = inter["k"][c * L:(c + 1) * L]
         assert (got_k != want_k).mean() < 0.05        # bf16 roundings of the fused epilogue
     plan.destroy()
+
+
+@pytest.mark.parametrize("epi", ["store", "gelu_tanh", "gated_residual", "qkv"])
+def test_repeat_runs_bit_identical(wf, epi):
+    """Ten launches of each GEMM epilogue (and of the LayerNorm) give the same bits:
+    a race in the stage ring or the double-buffered accumulator (a slot reused
+    early, an epilogue reading a tile the MMAs are overwriting) would show as
+    run-to-run differences.  Shapes of several tiles per cluster."""
+    dev = "cuda"
+    F, gh, gw, W, Hh, H, D = 2, 10, 26, 4, 1, 4, 128     # T = 2080, N = 1536 for qkv
+    L, T, C = F * gh * gw, W * F * gh * gw, 512
+    x = wi.bf16_normal((T, C), 31, wi.STREAM_X).to(dev)
+    plan = wf.Plan(L, W, Hh, H, D).set_rope(F, gh, gw)
+    outs = []
+    if epi == "qkv":
+        w_qkv = wi.bf16_weight(3 * H * D, C, 31).to(dev)
+        gq, gk = (t.to(dev) for t in wi.gains(H, D, 31))
+        q_out = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+        kc = torch.zeros((W + Hh, L, H, D), dtype=torch.bfloat16, device=dev)
+        vc = torch.zeros_like(kc)
+        for _ in range(10):
+            wf.wf_qkv_proj_norm_rope_append(plan, 3, x, w_qkv, None, gq, gk, q_out, kc, vc)
+            outs.append(torch.cat([q_out.view(-1), kc.view(-1), vc.view(-1)]).view(torch.int16)
+                        .clone())
+    else:
+        N = 1280
+        w = wi.bf16_weight(N, C, 32).to(dev)
+        b = wi.f32_vector((N,), 0.5, 32, wi.STREAM_BIAS).to(dev)
+        gate = wi.f32_vector((W, N), 1.0, 32, wi.STREAM_MOD).to(dev)
+        resid = wi.bf16_normal((T, N), 32, wi.STREAM_V).to(dev)
+        y = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
+        code = {"store": wf.WF_EPI_STORE, "gelu_tanh": wf.WF_EPI_GELU_TANH,
+                "gated_residual": wf.WF_EPI_GATED_RESIDUAL}[epi]
+        gr = epi == "gated_residual"
+        for _ in range(10):
+            wf.wf_linear(plan, x, w, y, b, code, gate if gr else None, resid if gr else None, L)
+            outs.append(y.view(torch.int16).clone())
+        mod = wi.f32_vector((2, W, C), 0.3, 33, wi.STREAM_MOD).to(dev)
+        h = torch.empty_like(x)
+        hs = []
+        for _ in range(10):
+            wf.wf_layer_norm_modulate(plan, x, mod[0], mod[1], L, h)
+            hs.append(h.view(torch.int16).clone())
+        assert all(torch.equal(hs[0], t) for t in hs[1:])
+    torch.cuda.synchronize()
+    assert wf.wf_sync_status(plan) == wf.WF_OK
+    assert all(torch.equal(outs[0], t) for t in outs[1:])
+    plan.destroy()
