@@ -1,7 +1,8 @@
 // attn_kernel.cu -- chunk-causal wave-round attention on sm_100a tensor cores.
 //
-// "Wave Forcing" (abstract): chunk-wise causal attention lets each chunk of the
-// wave read earlier, cleaner chunks before their denoising is complete.  For
+// "Wave Forcing" (abstract): with chunk-wise causal attention a chunk of the wave
+// can use the chunks ahead of it, which are less noisy, while those are still
+// being denoised.  For
 // query chunk c the visible keys are every token of the valid history chunks
 // and of wave chunks 0..c; inside a chunk attention is bidirectional.  Visible
 // keys therefore form whole chunks, so masking is decided per key tile: fully

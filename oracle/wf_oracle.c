@@ -38,9 +38,10 @@
  *       concatenation of key chunks, each tagged with its absolute chunk id.
  *       Key j is visible to query n exactly when chunk_id(j) <= chunk_id(n):
  *       later chunks see earlier (cleaner) chunks and all of their own chunk,
- *       never a later chunk ("Wave Forcing" abstract: chunk-wise causal
- *       attention reaching earlier, cleaner chunks before their denoising is
- *       complete).  s_j = q.k_j / sqrt(D); p = softmax over visible j;
+ *       never a later chunk ("Wave Forcing" abstract: under chunk-wise causal
+ *       attention a chunk uses the less noisy chunks ahead of it while they
+ *       are still being denoised).  s_j = q.k_j / sqrt(D); p = softmax over
+ *       visible j;
  *       O = sum_j p_j v_j; lse = m + log(sum_j exp(s_j - m)).
  *
  *   wfo_e4m3_encode / wfo_e4m3_decode
