@@ -395,3 +395,81 @@ def test_repeat_runs_bit_identical(wf, epi):
     assert wf.wf_sync_status(plan) == wf.WF_OK
     assert all(torch.equal(outs[0], t) for t in outs[1:])
     plan.destroy()
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 32, 8), (257, 32, 8), (3, 64, 2056), (511, 256, 72)])
+def test_linear_edge_shapes(wf, M, N, K):
+    """Degenerate and ragged GEMM shapes: one row, the smallest N and K the call
+    accepts, one row past a 256-row tile, a K of 32 slices plus 8, a single column
+    tile with M one short of two tiles."""
+    dev = "cuda"
+    seed = 3 * M + N + K
+    x = wi.bf16_normal((M, K), seed, wi.STREAM_X)
+    w = wi.bf16_weight(N, K, seed)
+    bias = wi.f32_vector((N,), 0.5, seed, wi.STREAM_BIAS)
+    gate = wi.f32_vector((1, N), 1.0, seed, wi.STREAM_MOD)
+    resid = wi.bf16_normal((M, N), seed, wi.STREAM_V)
+    plan = wf.Plan(32, 1, 0, 1, 64)
+    for epi, code in (("store", wf.WF_EPI_STORE), ("gelu_tanh", wf.WF_EPI_GELU_TANH),
+                      ("gated_residual", wf.WF_EPI_GATED_RESIDUAL)):
+        y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=dev)
+        gr = epi == "gated_residual"
+        wf.wf_linear(plan, x.to(dev), w.to(dev), y, bias.to(dev), code,
+                     gate.to(dev) if gr else None, resid.to(dev) if gr else None, M)
+        torch.cuda.synchronize()
+        assert wf.wf_sync_status(plan) == wf.WF_OK
+        ref = ob.linear_f64(_bits(x), _bits(w), bias.numpy(), epi, gate.numpy() if gr else None,
+                            _bits(resid) if gr else None, M)
+        S = _abs_sum(x, w) * (np.abs(gate.numpy().astype(np.float64)) if gr else 1.0)
+        _assert_gemm_close(_bits(y), ref, S, "linear %s %dx%dx%d" % (epi, M, N, K))
+    plan.destroy()
+
+
+def test_qkv_first_round_with_history_slots(wf):
+    """Round 0 of a ring with history slots (no history visible yet): the fused
+    projection writes the wave's chunks to slots 0..W-1 with t = c*F + f and
+    leaves the history slots alone."""
+    dev = "cuda"
+    F, gh, gw, W, Hh, H, D, C = 1, 4, 9, 2, 3, 1, 128, 128
+    L, T, R = F * gh * gw, W * F * gh * gw, W + Hh
+    x = wi.bf16_normal((T, C), 41, wi.STREAM_X)
+    w_qkv = wi.bf16_weight(3 * H * D, C, 41)
+    gq, gk = wi.gains(H, D, 41)
+    plan = wf.Plan(L, W, Hh, H, D).set_rope(F, gh, gw)
+    q_out = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+    kc = torch.full((R, L, H, D), -5.0, dtype=torch.bfloat16, device=dev)
+    vc = torch.full_like(kc, -5.0)
+    wf.wf_qkv_proj_norm_rope_append(plan, 0, x.to(dev), w_qkv.to(dev), None, gq.to(dev),
+                                    gk.to(dev), q_out, kc, vc)
+    torch.cuda.synchronize()
+    assert wf.wf_sync_status(plan) == wf.WF_OK
+    pos = oracle.positions(0, W, F, gh, gw)
+    _, _, _, q64, k64, v64 = ob.qkv_project_append(_bits(x), _bits(w_qkv), None, pos, gq.numpy(),
+                                                   gk.numpy(), H, D, want_f64=True)
+    y = ob.linear_f64(_bits(x), _bits(w_qkv)).reshape(T, 3, H, D)
+    S = _abs_sum(x, w_qkv).reshape(T, 3, H, D)
+    got_k = np.concatenate([_bits(kc[c]) for c in range(W)])
+    _assert_qk_close(_bits(q_out), q64, y[:, 0], S[:, 0], gq, "q round 0")
+    _assert_qk_close(got_k, k64, y[:, 1], S[:, 1], gk, "k round 0")
+    for slot in range(W, R):
+        assert (kc[slot].float() == -5.0).all() and (vc[slot].float() == -5.0).all()
+    plan.destroy()
+
+
+def test_layer_norm_single_row_and_group(wf):
+    """One row of 64 channels around a common offset, one modulation group."""
+    dev = "cuda"
+    x = (wi.bf16_normal((1, 64), 5, wi.STREAM_X).float() * 0.5 + 3.0).to(torch.bfloat16)
+    shift = wi.f32_vector((1, 64), 0.5, 5, wi.STREAM_MOD)
+    scale = wi.f32_vector((1, 64), 0.5, 5, wi.STREAM_BIAS)
+    plan = wf.Plan(32, 1, 0, 1, 64)
+    y = torch.empty((1, 64), dtype=torch.bfloat16, device=dev)
+    wf.wf_layer_norm_modulate(plan, x.to(dev), shift.to(dev), scale.to(dev), 1, y)
+    torch.cuda.synchronize()
+    ref = ob.layer_norm_modulate_f64(_bits(x), shift.numpy(), scale.numpy(), 1)
+    xh = ob.layer_norm_modulate_f64(_bits(x), np.zeros(64, np.float32), np.zeros(64, np.float32), 1)
+    mag = np.abs(xh * (1.0 + scale.numpy())) + np.abs(shift.numpy())
+    r_bf = oracle.bf16_to_f64(oracle.f64_to_bf16(ref))
+    tol = bf16_quantum(r_bf) * 1.0000001 + 2.0 ** -18 * mag   # the bar of the main LN test
+    assert (np.abs(_f64(y.float()) - ref) <= tol).all()
+    plan.destroy()

@@ -25,11 +25,11 @@ def wf():
     return mod
 
 
-@pytest.mark.parametrize("world", [1, 2, 3, 5])
-def test_emulated_ranks_equal_single_wave(wf, world):
+@pytest.mark.parametrize("world,Hh", [(1, 2), (2, 2), (3, 2), (5, 2), (5, 0), (2, 0)])
+def test_emulated_ranks_equal_single_wave(wf, world, Hh):
     from chunk_causal_dit_b200.wave_parallel import LibwfKernels, WaveParallelRound
     dev = "cuda"
-    F, gh, gw, W, Hh, H, D = 2, 6, 25, 5, 2, 2, 128
+    F, gh, gw, W, H, D = 2, 6, 25, 5, 2, 128
     L = F * gh * gw
     R = Hh + W
     rounds = 2
