@@ -16,14 +16,16 @@
 //    (columns of C).  The leader issues tcgen05.mma.cta_group::2 with M = 256,
 //    N = 256, K = 16; each SM reads half of the B tile, so a stage is 32 KB per
 //    SM for 512 tensor cycles of work.
-//  * A 6-stage ring of 64-deep K slices (one 128-byte swizzle row of bf16),
-//    filled by TMA; both CTAs' copies complete on the leader's barriers, the
-//    leader's commits release the stage in both CTAs.
+//  * A ring of 64-deep K slices (one 128-byte swizzle row of bf16; 6 stages, 5
+//    with the QKV epilogue's RoPE tables), filled by TMA; both CTAs' copies
+//    complete on the leader's barriers, the leader's commits release the stage
+//    in both CTAs.
 //  * Two 256-column fp32 accumulators in TMEM (all 512 columns): the epilogue of
 //    tile i reads one while the MMAs of tile i + 1 fill the other.
 //  * Eight epilogue warps per CTA: warp w reads TMEM lane quarter w % 4 (the
 //    lanes a warp may access) and one 128-column half of the tile; each thread
-//    owns one row of C.
+//    owns one row of C, and the warp moves its global loads and stores through
+//    a staging buffer in shared memory so that they are coalesced.
 //  * Tiles are dealt statically: cluster c takes tiles c, c + clusters, ...,
 //    numbered with the column tile fastest, so the clusters working at one time
 //    share a few row blocks of A (and all of B) in L2.
