@@ -840,6 +840,172 @@ def run_block_round_loop(args, rank, world, local):
     }
 
 
+def run_wp_block(args, rank, world, local):
+    """Wave Parallelism on the whole DiT block: every rank runs the block on its
+    own chunks (LayerNorm, fused QKV projection, K/V delivery, attention, output
+    projection, feed-forward); the round advances every step.  Under torchrun
+    the delivery is NCCL and the step time the device-timed max over ranks; in
+    one process the ranks run one after another on the one GPU, each half of a
+    rank's block (before and after the delivery) is timed, and the step time is
+    *projected* as the slowest rank's before + delivery (at the peer-copy
+    bandwidth) + after, next to the single-GPU block measured in the same process."""
+    import torch
+    from chunk_causal_dit_b200 import wf
+    from chunk_causal_dit_b200.wave_parallel import LibwfKernels, WaveParallelRound
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = make_group(world, "nccl")
+    w = wi.WORKLOADS[args.workload]
+    hidden, ffn = wi.BLOCK_WIDTHS[w.H * w.D]
+    emulate = world == 1
+    n_ranks = args.wp if emulate else world
+    if not 1 <= n_ranks <= w.n_wave:
+        raise SystemExit("Wave Parallelism needs 1..%d ranks" % w.n_wave)
+    b = wi.block_inputs(w, hidden, ffn, seed=0)
+    wts = {k: getattr(b, k).to(dev) for k in ("w_qkv", "b_qkv", "w_o", "b_o", "w_1", "b_1",
+                                              "w_2", "b_2")}
+    mod = b.mod.to(dev)
+    kern = LibwfKernels(b.gamma_q.to(dev), b.gamma_k.to(dev))
+    hk, hv = wi.history_prefill(w, seed=0)
+    r0 = w.n_hist
+    mine = list(range(n_ranks)) if emulate else [rank]
+
+    def setup(wp):
+        t = {"h": torch.empty((wp.rows, hidden), dtype=torch.bfloat16, device=dev),
+             "q_out": torch.empty((wp.rows, w.H, w.D), dtype=torch.bfloat16, device=dev),
+             "o": torch.empty((wp.rows, w.H, w.D), dtype=torch.bfloat16, device=dev),
+             "f": torch.empty((wp.rows, ffn), dtype=torch.bfloat16, device=dev),
+             "k_cache": torch.empty(wp.ring_shape(), dtype=torch.bfloat16, device=dev),
+             "v_cache": torch.empty(wp.ring_shape(), dtype=torch.bfloat16, device=dev),
+             "x0": b.x[wp.c0 * w.L:wp.c1 * w.L].to(dev)}
+        t["x"] = torch.empty_like(t["x0"])
+        wp.prefill_history(r0, [(r0 - w.n_hist + j, hk[j].to(dev), hv[j].to(dev))
+                                for j in range(w.n_hist)], t["k_cache"], t["v_cache"])
+        return t
+
+    wps, ten = {}, {}
+    for k in mine:
+        kw = {"world": n_ranks, "rank": k} if emulate else {}
+        wps[k] = WaveParallelRound(w.L, w.n_wave, w.n_hist, w.H, w.D, (w.F, w.gh, w.gw), kern,
+                                   **kw)
+        ten[k] = setup(wps[k])
+    stream = torch.cuda.current_stream(dev)
+
+    def step(r, ev=None):
+        for k in mine:
+            ten[k]["x"].copy_(ten[k]["x0"])
+        if not emulate:
+            wp, t = wps[rank], ten[rank]
+            wp.run_block(r, t["x"], wts, mod, t)
+            return
+        ms = {k: wps[k].mod_rows(mod) for k in mine}
+        for i, k in enumerate(mine):
+            if ev is not None:
+                ev[i][0].record(stream)
+            wps[k].norm_and_qkv(r, ten[k]["x"], wts, ms[k], ten[k])
+            if ev is not None:
+                ev[i][1].record(stream)
+        for k in mine:                       # stand-in for the NCCL delivery (not timed)
+            for src, g in wps[k].incoming(r):
+                for c in ("k_cache", "v_cache"):
+                    ten[k][c][wps[k].slot(g)].copy_(ten[src][c][wps[src].slot(g)])
+        for i, k in enumerate(mine):
+            if ev is not None:
+                ev[i][2].record(stream)
+            wps[k].attention_and_rest(r, ten[k]["x"], wts, ms[k], ten[k])
+            if ev is not None:
+                ev[i][3].record(stream)
+
+    rnd = r0
+    for _ in range(args.warmup):
+        step(rnd)
+        rnd += 1
+    torch.cuda.synchronize(dev)
+    steps = args.steps
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in mine]
+           for _ in range(steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dist, dev)
+    torch.cuda.synchronize(dev)
+    start.record(stream)
+    for i in range(steps):
+        step(rnd, evs[i] if emulate else None)
+        rnd += 1
+    stop.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    for k in mine:
+        st = wf.wf_sync_status(wps[k].plan)
+        if st != wf.WF_OK:
+            raise SystemExit("wave parallel block: device status %d (%s)"
+                             % (st, wf.status_string(st)))
+    ms_step = allreduce_max(dist, start.elapsed_time(stop), dev) / steps
+    full = wf.Plan(w.L, w.n_wave, w.n_hist, w.H, w.D)
+    flops_step = block_flops(w, hidden, ffn, wf.wf_useful_flops(full, r0))
+    full.destroy()
+    line = None
+    if rank == 0:
+        line = {
+            "metric": "DiT block over the wave, useful TFLOP/s (Wave Parallelism, %d ranks)"
+                      % n_ranks,
+            "unit": "TFLOP/s", "n_gpus": world, "steps": steps, "warmup": args.warmup,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded bf16; random-init block weights)",
+            "config": {"workload": w.name, "hidden": hidden, "ffn": ffn,
+                       "wave_parallel_ranks": n_ranks,
+                       "parallelism": "wave-parallel %d (one-way K/V delivery, NCCL p2p)"
+                       % n_ranks},
+        }
+        if not emulate:
+            line.update({"value": round(flops_step / (ms_step * 1e-3) / 1e12, 3),
+                         "ms_per_step": round(ms_step, 5), "projected": False})
+        else:
+            chunk_bytes = 2 * w.L * w.H * w.D * 2
+            per = []
+            for i, k in enumerate(mine):
+                wp = wps[k]
+                pre = statistics.mean(e[i][0].elapsed_time(e[i][1]) for e in evs)
+                post = statistics.mean(e[i][2].elapsed_time(e[i][3]) for e in evs)
+                recv = len(wp.incoming(r0)) * chunk_bytes
+                per.append({"rank": k, "chunks": [wp.c0, wp.c1], "norm_qkv_ms": round(pre, 5),
+                            "attention_and_rest_ms": round(post, 5), "recv_bytes": recv,
+                            "recv_ms_at_peer_copy": round(recv / (PEER_COPY_GBS * 1e6), 5)})
+            proj = max(p["norm_qkv_ms"] + p["recv_ms_at_peer_copy"] + p["attention_and_rest_ms"]
+                       for p in per)
+            one = WaveParallelRound(w.L, w.n_wave, w.n_hist, w.H, w.D, (w.F, w.gh, w.gw), kern,
+                                    world=1, rank=0)
+            t1 = setup(one)
+            for i in range(3):
+                t1["x"].copy_(t1["x0"])
+                one.run_block(r0 + i, t1["x"], wts, mod, t1)
+            torch.cuda.synchronize(dev)
+            a, c = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for i in range(steps):
+                t1["x"].copy_(t1["x0"])
+                one.run_block(r0 + 3 + i, t1["x"], wts, mod, t1)
+            c.record(stream)
+            torch.cuda.synchronize(dev)
+            single = a.elapsed_time(c) / steps
+            one.destroy()
+            line.update({
+                "value": round(flops_step / (proj * 1e-3) / 1e12, 3),
+                "ms_per_step": round(proj, 5), "projected": True,
+                "projection": "max over ranks of (LayerNorm + QKV, incoming K/V at %.0f GB/s peer "
+                              "copy, attention + the rest of the block), each rank's kernels timed "
+                              "alone on one B200" % PEER_COPY_GBS,
+                "per_rank": per,
+                "single_gpu_ms_per_step": round(single, 5),
+                "speedup_projected": round(single / proj, 3),
+            })
+    for wp in wps.values():
+        wp.destroy()
+    if dist is not None:
+        dist.destroy_process_group()
+    return line
+
+
 def run_round_loop(args, rank, world, local):
     """Full rounds of a multi-layer workload: every round runs, layer after layer,
     the append and the attention of each layer on that layer's own ring, then
@@ -1069,7 +1235,8 @@ def main():
     ap.add_argument("--attn", default="bf16", choices=["bf16", "fp8qk"],
                     help="attention variant: bf16 (default) or E4M3 Q.K^T with bf16 P.V")
     ap.add_argument("--blocks", action="store_true",
-                    help="with a multi-layer workload: every layer runs the whole DiT block")
+                    help="with a multi-layer workload: every layer runs the whole DiT block; "
+                         "with --wp: Wave Parallelism on the whole block")
     ap.add_argument("--wp", type=int, default=0,
                     help="Wave Parallelism: under torchrun, split the wave over the ranks; "
                          "in one process, emulate N ranks on the one GPU (projected time)")
@@ -1083,6 +1250,8 @@ def main():
     rank, world, local = dist_setup(args.gpus)
     if args.impl == "reference":
         line = run_reference(args, rank, world)
+    elif args.wp and args.blocks:
+        line = run_wp_block(args, rank, world, local)
     elif args.wp:
         line = run_wp(args, rank, world, local)
     elif wi.WORKLOADS[args.workload].layers > 1 and args.blocks:

@@ -93,6 +93,17 @@ class LibwfKernels:
     def attention(self, plan, round_: int, q_out, k_cache, v_cache, o) -> None:
         self.wf.wf_chunk_causal_attn(plan, round_, q_out, k_cache, v_cache, o, None)
 
+    # the DiT block's calls (run_block)
+    def layer_norm(self, plan, x, shift, scale, rows_per_group, y) -> None:
+        self.wf.wf_layer_norm_modulate(plan, x, shift, scale, rows_per_group, y)
+
+    def qkv(self, plan, round_: int, h, w_qkv, b_qkv, q_out, k_cache, v_cache) -> None:
+        self.wf.wf_qkv_proj_norm_rope_append(plan, round_, h, w_qkv, b_qkv, self.gq, self.gk,
+                                             q_out, k_cache, v_cache)
+
+    def linear(self, plan, x, w, y, bias, epilogue, gate, resid, rows_per_group) -> None:
+        self.wf.wf_linear(plan, x, w, y, bias, epilogue, gate, resid, rows_per_group)
+
 
 def libwf_plan(L: int, n_wave: int, n_hist: int, H: int, D: int, rope: Tuple[int, int, int]):
     from . import wf
@@ -195,6 +206,51 @@ class WaveParallelRound:
         self.kernels.append(self.plan, r, q, k, v, q_out, k_cache, v_cache)
         self.exchange(round_, k_cache, v_cache)
         self.kernels.attention(self.plan, r, q_out, k_cache, v_cache, o)
+
+    def run_block(self, round_: int, x, w, mod, buf) -> None:
+        """One DiT block of round `round_` for this rank's chunks (the whole block
+        runs on the rank's rows; the only exchange is the K/V delivery between the
+        QKV projection and the attention):
+
+        * x [rows, C]: the rank's residual stream, updated in place;
+        * w: dict of the block's weights (w_qkv, b_qkv, w_o, b_o, w_1, b_1, w_2,
+          b_2), as ``wf_linear`` / ``wf_qkv_proj_norm_rope_append`` take them;
+        * mod [6, W, C]: the whole wave's modulation rows (shift, scale and gate
+          of the attention half, then of the feed-forward half); the rank uses
+          rows c0..c1-1;
+        * buf: dict of work buffers h [rows, C], q_out and o [rows, H, D], f
+          [rows, F], and the ring k_cache, v_cache (ring_shape()).
+        The kernels object needs ``layer_norm``, ``qkv``, ``attention`` and
+        ``linear`` (as ``LibwfKernels``)."""
+        m = self.mod_rows(mod)
+        self.norm_and_qkv(round_, x, w, m, buf)
+        self.exchange(round_, buf["k_cache"], buf["v_cache"])
+        self.attention_and_rest(round_, x, w, m, buf)
+
+    def mod_rows(self, mod):
+        """This rank's six modulation row blocks of a wave's table [6, W, C]."""
+        return [mod[i, self.c0:self.c1] for i in range(6)]
+
+    def norm_and_qkv(self, round_: int, x, w, m, buf) -> None:
+        """The block before the delivery: LayerNorm + modulation and the QKV
+        projection, whose epilogue appends this rank's K/V to its ring."""
+        k, plan = self.kernels, self.plan
+        k.layer_norm(plan, x, m[0], m[1], self.L, buf["h"])
+        k.qkv(plan, round_ + self.c0, buf["h"], w["w_qkv"], w["b_qkv"], buf["q_out"],
+              buf["k_cache"], buf["v_cache"])
+
+    def attention_and_rest(self, round_: int, x, w, m, buf) -> None:
+        """The block after the delivery: attention, output projection, norm and
+        feed-forward layers (m: the rank's six modulation row blocks)."""
+        from .wf import WF_EPI_GATED_RESIDUAL, WF_EPI_GELU_TANH
+        k, plan, L = self.kernels, self.plan, self.L
+        r = round_ + self.c0
+        k.attention(plan, r, buf["q_out"], buf["k_cache"], buf["v_cache"], buf["o"])
+        o2 = buf["o"].view(self.rows, self.H * self.D)
+        k.linear(plan, o2, w["w_o"], x, w["b_o"], WF_EPI_GATED_RESIDUAL, m[2], x, L)
+        k.layer_norm(plan, x, m[3], m[4], L, buf["h"])
+        k.linear(plan, buf["h"], w["w_1"], buf["f"], w["b_1"], WF_EPI_GELU_TANH, None, None, 1)
+        k.linear(plan, buf["f"], w["w_2"], x, w["b_2"], WF_EPI_GATED_RESIDUAL, m[5], x, L)
 
     def prefill_history(self, round_: int, history: Sequence[Tuple[int, torch.Tensor, torch.Tensor]],
                         k_cache, v_cache) -> None:

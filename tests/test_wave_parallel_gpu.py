@@ -93,3 +93,76 @@ def test_emulated_ranks_equal_single_wave(wf, world, Hh):
             assert torch.equal(got, ref), "world %d rank %d round %d" % (world, wp.rank, r)
     for wp in ranks:
         wp.destroy()
+
+
+@pytest.mark.parametrize("world", [2, 5])
+def test_emulated_ranks_run_the_block_like_one_gpu(wf, world):
+    """The whole DiT block per rank (LayerNorm, fused QKV projection, delivery,
+    attention, output projection, feed-forward), ranks emulated one after another
+    with device copies for the delivery: every rank's residual rows equal the
+    single-GPU block's, bit for bit, over two rounds.  (Each GEMM element sums K
+    in the same order whatever the row tiling; LayerNorm is per row; the
+    attention visits the same key tiles.)"""
+    from chunk_causal_dit_b200.wave_parallel import LibwfKernels, WaveParallelRound
+    dev = "cuda"
+    F, gh, gw, W, Hh, H, D, C, FF = 2, 6, 25, 5, 2, 2, 128, 256, 512
+    L, T, R = F * gh * gw, W * F * gh * gw, Hh + W
+    s = 17
+    w = {"w_qkv": wi.bf16_weight(3 * H * D, C, s, 1), "w_o": wi.bf16_weight(C, H * D, s, 2),
+         "w_1": wi.bf16_weight(FF, C, s, 3), "w_2": wi.bf16_weight(C, FF, s, 4),
+         "b_qkv": wi.f32_vector((3 * H * D,), 0.02, s, wi.STREAM_BIAS, 1),
+         "b_o": wi.f32_vector((C,), 0.02, s, wi.STREAM_BIAS, 2),
+         "b_1": wi.f32_vector((FF,), 0.02, s, wi.STREAM_BIAS, 3),
+         "b_2": wi.f32_vector((C,), 0.02, s, wi.STREAM_BIAS, 4)}
+    w = {k: t.to(dev) for k, t in w.items()}
+    mod = wi.f32_vector((6, W, C), 0.1, s, wi.STREAM_MOD).to(dev)
+    gq, gk = (t.to(dev) for t in wi.gains(H, D, s))
+    xs = [wi.bf16_normal((T, C), s + i, wi.STREAM_X).to(dev) for i in range(2)]
+    hk = wi.bf16_normal((Hh, L, H, D), s, 3).to(dev)
+    hv = wi.bf16_normal((Hh, L, H, D), s, 4).to(dev)
+    kern = LibwfKernels(gq, gk)
+    r0 = Hh
+
+    def buffers(rows, ring_shape):
+        return {"h": torch.empty((rows, C), dtype=torch.bfloat16, device=dev),
+                "q_out": torch.empty((rows, H, D), dtype=torch.bfloat16, device=dev),
+                "o": torch.empty((rows, H, D), dtype=torch.bfloat16, device=dev),
+                "f": torch.empty((rows, FF), dtype=torch.bfloat16, device=dev),
+                "k_cache": torch.zeros(ring_shape, dtype=torch.bfloat16, device=dev),
+                "v_cache": torch.zeros(ring_shape, dtype=torch.bfloat16, device=dev)}
+
+    def prefill(wp, buf):
+        wp.prefill_history(r0, [(r0 - Hh + j, hk[j], hv[j]) for j in range(Hh)],
+                           buf["k_cache"], buf["v_cache"])
+
+    one = WaveParallelRound(L, W, Hh, H, D, (F, gh, gw), kern, world=1, rank=0)
+    b1 = buffers(one.rows, one.ring_shape())
+    prefill(one, b1)
+    ranks = [WaveParallelRound(L, W, Hh, H, D, (F, gh, gw), kern, world=world, rank=k)
+             for k in range(world)]
+    bufs = [buffers(wp.rows, wp.ring_shape()) for wp in ranks]
+    for wp, b in zip(ranks, bufs):
+        prefill(wp, b)
+    for i in range(2):
+        r = r0 + i
+        X1 = xs[i].clone()
+        one.run_block(r, X1, w, mod, b1)
+        Xs = [xs[i][wp.c0 * L:wp.c1 * L].clone() for wp in ranks]
+        ms = [wp.mod_rows(mod) for wp in ranks]
+        for wp, b, X, m in zip(ranks, bufs, Xs, ms):
+            wp.norm_and_qkv(r, X, w, m, b)
+        for wp, b in zip(ranks, bufs):                       # the one-way delivery
+            for src, g in wp.incoming(r):
+                sb = bufs[src]
+                b["k_cache"][wp.slot(g)].copy_(sb["k_cache"][ranks[src].slot(g)])
+                b["v_cache"][wp.slot(g)].copy_(sb["v_cache"][ranks[src].slot(g)])
+        for wp, b, X, m in zip(ranks, bufs, Xs, ms):
+            wp.attention_and_rest(r, X, w, m, b)
+        torch.cuda.synchronize()
+        for wp, X in zip(ranks, Xs):
+            assert wf.wf_sync_status(wp.plan) == wf.WF_OK
+            ref = X1[wp.c0 * L:wp.c1 * L]
+            assert torch.equal(X.view(torch.int16), ref.view(torch.int16)), \
+                "world %d rank %d round %d" % (world, wp.rank, r)
+    for wp in ranks + [one]:
+        wp.destroy()
