@@ -1,11 +1,12 @@
 """Wave Parallelism host logic on CPU: the chunk partition, and the one-way K/V
 exchange between gloo ranks over consecutive rounds.
 
-The exchange test runs each rank's append and attention with the oracle (CPU
-stand-ins defined here, test-only), so every difference from the expected
-output is a difference in what the rank's ring holds: which chunks it received,
-into which slots, in which round.  The expectation is the oracle's own round,
-computed in one process from absolute chunk ids with no ring at all.
+The exchange tests run each rank's kernels with the oracle (CPU stand-ins
+defined here, test-only), so every difference from the expected output is a
+difference in what the rank's ring holds: which chunks it received, into
+which slots, in which round.  The expectation is the oracle's own round (the
+append and attention, or the whole DiT block of oracle/block.py), computed in
+one process from absolute chunk ids with no ring at all.
 """
 import itertools
 import os
@@ -104,6 +105,58 @@ class OracleKernels:
         o_out.copy_(wi.from_bits(o.f64_to_bf16(ref)).view(o_out.shape))
 
 
+class OracleBlockKernels(OracleKernels):
+    """The block's calls on the oracle (test-only, CPU), with the GPU calls'
+    conventions: the QKV projection writes q_out and the ring slots g mod R of the
+    plan's chunks; linear layers may write their output over their residual."""
+
+    def __init__(self, gq, gk):
+        super().__init__(gq, gk)
+        import oracle.block as ob
+        from chunk_causal_dit_b200 import wf
+        self.ob = ob
+        self.epi = {wf.WF_EPI_STORE: "store", wf.WF_EPI_GELU_TANH: "gelu_tanh",
+                    wf.WF_EPI_GATED_RESIDUAL: "gated_residual"}
+
+    def layer_norm(self, plan, x, shift, scale, rpg, y):
+        wi = self.wi
+        y.copy_(wi.from_bits(self.ob.layer_norm_modulate(wi.bits(x), shift.numpy(),
+                                                          scale.numpy(), rpg)))
+
+    def qkv(self, plan, r, h, w_qkv, b_qkv, q_out, kc, vc):
+        wi = self.wi
+        pos = self.o.positions(r, plan.W, SHAPE["F"], SHAPE["gh"], SHAPE["gw"])
+        q, k, v = self.ob.qkv_project_append(wi.bits(h), wi.bits(w_qkv), b_qkv.numpy(), pos,
+                                             self.gq, self.gk, plan.H, plan.D)
+        q_out.copy_(wi.from_bits(q))
+        L = plan.L
+        for c in range(plan.W):
+            s = (r + c) % plan.R
+            kc[s].copy_(wi.from_bits(k[c * L:(c + 1) * L]))
+            vc[s].copy_(wi.from_bits(v[c * L:(c + 1) * L]))
+
+    def linear(self, plan, x, w, y, bias, epilogue, gate, resid, rpg):
+        wi = self.wi
+        out = self.ob.linear(wi.bits(x), wi.bits(w), None if bias is None else bias.numpy(),
+                             self.epi[epilogue], None if gate is None else gate.numpy(),
+                             None if resid is None else wi.bits(resid), rpg)
+        y.copy_(wi.from_bits(out))
+
+
+BLOCK = dict(C=SHAPE["H"] * SHAPE["D"], FF=192)
+
+
+def _block_weights(seed=9):
+    from chunk_causal_dit_b200 import inputs as wi
+    C, FF, HD = BLOCK["C"], BLOCK["FF"], SHAPE["H"] * SHAPE["D"]
+    return {"w_qkv": wi.bf16_weight(3 * HD, C, seed, 1), "w_o": wi.bf16_weight(C, HD, seed, 2),
+            "w_1": wi.bf16_weight(FF, C, seed, 3), "w_2": wi.bf16_weight(C, FF, seed, 4),
+            "b_qkv": wi.f32_vector((3 * HD,), 0.02, seed, wi.STREAM_BIAS, 1),
+            "b_o": wi.f32_vector((C,), 0.02, seed, wi.STREAM_BIAS, 2),
+            "b_1": wi.f32_vector((FF,), 0.02, seed, wi.STREAM_BIAS, 3),
+            "b_2": wi.f32_vector((C,), 0.02, seed, wi.STREAM_BIAS, 4)}
+
+
 def _plan_factory(L, n, hist, H, D, rope):
     return SimpleNamespace(L=L, W=n, Hh=hist, H=H, D=D, R=hist + n)
 
@@ -197,3 +250,73 @@ def test_exchange_over_gloo_matches_single_wave(world, W, Hh):
             want = expected[i][c0 * L:c1 * L]
             assert np.array_equal(res[i], want), "rank %d round %d" % (rank, i)
     assert covered == list(range(W))
+
+
+def _rank_block_main(rank, world, port, W, Hh, r0, rounds, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    from chunk_causal_dit_b200 import inputs as wi
+    from chunk_causal_dit_b200.wave_parallel import WaveParallelRound
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        L, xs, hk, hv, gq, gk = _inputs(W, Hh, rounds)
+        H, D, C, FF = SHAPE["H"], SHAPE["D"], BLOCK["C"], BLOCK["FF"]
+        w = _block_weights()
+        mod = wi.f32_vector((6, W, C), 0.1, 9, wi.STREAM_MOD)
+        wp = WaveParallelRound(L, W, Hh, H, D, (SHAPE["F"], SHAPE["gh"], SHAPE["gw"]),
+                               OracleBlockKernels(gq, gk), plan_factory=_plan_factory)
+        buf = {"h": torch.empty((wp.rows, C), dtype=torch.bfloat16),
+               "q_out": torch.empty((wp.rows, H, D), dtype=torch.bfloat16),
+               "o": torch.empty((wp.rows, H, D), dtype=torch.bfloat16),
+               "f": torch.empty((wp.rows, FF), dtype=torch.bfloat16),
+               "k_cache": torch.zeros(wp.ring_shape(), dtype=torch.bfloat16),
+               "v_cache": torch.zeros(wp.ring_shape(), dtype=torch.bfloat16)}
+        wp.prefill_history(r0, [(r0 - Hh + j, hk[j], hv[j]) for j in range(Hh)],
+                           buf["k_cache"], buf["v_cache"])
+        res = []
+        for i in range(rounds):
+            x = _block_x(W, L, i)[wp.c0 * L:wp.c1 * L].clone()
+            wp.run_block(r0 + i, x, w, mod, buf)
+            res.append(wi.bits(x))
+        out[rank] = (wp.c0, wp.c1, res)
+    finally:
+        dist.destroy_process_group()
+
+
+def _block_x(W, L, i):
+    from chunk_causal_dit_b200 import inputs as wi
+    return wi.bf16_normal((W * L, BLOCK["C"]), 40 + i, wi.STREAM_X)
+
+
+@pytest.mark.parametrize("world,W,Hh", [(2, 3, 1), (3, 4, 2)])
+def test_block_exchange_over_gloo_matches_the_oracle_block(world, W, Hh):
+    """run_block on gloo ranks (the exchange posted between the QKV projection and
+    the attention) against oracle.block.block_forward of the whole wave, over two
+    rounds (the second reads history delivered in the first)."""
+    import oracle
+    import oracle.block as ob
+    from chunk_causal_dit_b200 import inputs as wi
+    r0, rounds = Hh, 2
+    port = _free_port()
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_rank_block_main, args=(world, port, W, Hh, r0, rounds, out),
+                       nprocs=world, join=True, start_method="spawn")
+    L, xs, hk, hv, gq, gk = _inputs(W, Hh, rounds)
+    H, D, C = SHAPE["H"], SHAPE["D"], BLOCK["C"]
+    w = _block_weights()
+    wts = {k: (wi.bits(t) if t.dtype == torch.bfloat16 else t.numpy()) for k, t in w.items()}
+    wts["gamma_q"], wts["gamma_k"] = gq.numpy(), gk.numpy()
+    mod = wi.f32_vector((6, W, C), 0.1, 9, wi.STREAM_MOD).numpy()
+    cache = oracle.OracleCache(L)
+    for j in range(Hh):
+        cache.put(r0 - Hh + j, wi.bits(hk[j]), wi.bits(hv[j]))
+    for i in range(rounds):
+        r = r0 + i
+        pos = oracle.positions(r, W, SHAPE["F"], SHAPE["gh"], SHAPE["gw"])
+        want, _ = ob.block_forward(wi.bits(_block_x(W, L, i)), wts, mod, pos, cache, r, W, Hh,
+                                   H, D, L)
+        for rank in range(world):
+            c0, c1, res = out[rank]
+            assert np.array_equal(res[i], want[c0 * L:c1 * L]), "rank %d round %d" % (rank, r)
