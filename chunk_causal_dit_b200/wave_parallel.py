@@ -28,10 +28,10 @@ Per layer, each rank:
 
 History chunks are wave chunk 0 of earlier rounds, the refresh chunk of the
 rank that owns chunk 0. They arrived then and stay in the ring.  The sends are
-issued before the sender's attention, so the delivery runs on the
-communication stream while the sender computes.  A receiver's attention waits
-for its whole exchange, its own sends included: point-to-point operations
-posted together complete together.
+posted right after the append, before the sender's attention.  The first rank
+receives nothing, so its attention overlaps its sends.  A receiver's attention
+waits for its whole exchange, its own sends included: point-to-point
+operations posted together complete together.
 
 This module computes nothing.  The append and the attention are libwf kernels
 (``LibwfKernels``). For the CPU tests of the exchange they are whatever
@@ -144,6 +144,7 @@ class WaveParallelRound:
         self.R = n_hist + self.c1                 # this rank's ring slots
         self.kernels = kernels
         self.plan = (plan_factory or libwf_plan)(L, self.n, n_hist + self.c0, H, D, rope)
+        self._pending = []                        # sends not yet waited for (see exchange)
 
     # ---- layout of the rank's tensors ----
     @property
@@ -190,19 +191,38 @@ class WaveParallelRound:
         return ops
 
     def exchange(self, round_: int, k_cache, v_cache) -> None:
+        """Post this round's sends and receives as one batch.  A rank that receives
+        nothing (the first rank) does not wait for its sends: its attention only
+        reads the slots being sent, so the delivery overlaps it; the sends are
+        waited for before the rank next writes its ring (``settle``).  A rank that
+        receives waits for the whole batch (sends and receives posted together
+        complete together; posting them as two batches would serialise the ranks)."""
         if self.world == 1:
             return
         if self.emulated:
             raise RuntimeError("an emulated rank has no process group to exchange over")
+        self.settle()
         ops = self.exchange_ops(round_, k_cache, v_cache)
-        if ops:
-            for work in dist.batch_isend_irecv(ops):
+        if not ops:
+            return
+        works = dist.batch_isend_irecv(ops)
+        if self.incoming(round_):
+            for work in works:
                 work.wait()
+        else:
+            self._pending = list(works)
+
+    def settle(self) -> None:
+        """Wait for sends still in flight (before the ring is written again)."""
+        for work in self._pending:
+            work.wait()
+        self._pending = []
 
     def run_layer(self, round_: int, q, k, v, q_out, k_cache, v_cache, o) -> None:
         """One layer of round `round_` for this rank's chunks: append, exchange,
         attention.  q, k, v, q_out, o: [rows, H, D]; k_cache, v_cache: ring_shape()."""
         r = round_ + self.c0
+        self.settle()
         self.kernels.append(self.plan, r, q, k, v, q_out, k_cache, v_cache)
         self.exchange(round_, k_cache, v_cache)
         self.kernels.attention(self.plan, r, q_out, k_cache, v_cache, o)
@@ -235,6 +255,7 @@ class WaveParallelRound:
         """The block before the delivery: LayerNorm + modulation and the QKV
         projection, whose epilogue appends this rank's K/V to its ring."""
         k, plan = self.kernels, self.plan
+        self.settle()
         k.layer_norm(plan, x, m[0], m[1], self.L, buf["h"])
         k.qkv(plan, round_ + self.c0, buf["h"], w["w_qkv"], w["b_qkv"], buf["q_out"],
               buf["k_cache"], buf["v_cache"])
@@ -261,5 +282,6 @@ class WaveParallelRound:
             v_cache[self.slot(g)].copy_(vv)
 
     def destroy(self) -> None:
+        self.settle()
         if hasattr(self.plan, "destroy"):
             self.plan.destroy()

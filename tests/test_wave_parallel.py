@@ -203,6 +203,7 @@ def _rank_main(rank, world, port, W, Hh, r0, rounds, out):
             o = torch.empty_like(q)
             wp.run_layer(r0 + i, q, k, v, q_out, kc, vc, o)
             res.append(wi.bits(o))
+        wp.destroy()                             # waits for sends still in flight
         out[rank] = (wp.c0, wp.c1, res)
     finally:
         dist.destroy_process_group()
@@ -279,6 +280,7 @@ def _rank_block_main(rank, world, port, W, Hh, r0, rounds, out):
             x = _block_x(W, L, i)[wp.c0 * L:wp.c1 * L].clone()
             wp.run_block(r0 + i, x, w, mod, buf)
             res.append(wi.bits(x))
+        wp.destroy()
         out[rank] = (wp.c0, wp.c1, res)
     finally:
         dist.destroy_process_group()
