@@ -119,3 +119,26 @@ def test_append_alternative_tiny_positions(wf):
                         x.gamma_k.numpy(), want_f64=True)
     check_append(w, 0, ref, (wi.bits(q_out.cpu()), wi.bits(kc.cpu()), wi.bits(vc.cpu())))
     plan.destroy()
+
+
+def test_append_in_place_q(wf):
+    """q_out may alias q (wf.h): the in-place call writes the same bits as the call
+    with a separate q_out, on a ragged wave with several blocks per token range."""
+    w = wi.Workload("inplace", 3, 128, 2, 6, 25, 3, 1)        # L = 300
+    x = wi.wave_inputs(w, seed=4)
+    dev = "cuda"
+    q, k, v = x.q.to(dev), x.k.to(dev), x.v.to(dev)
+    gq, gk = x.gamma_q.to(dev), x.gamma_k.to(dev)
+    plan = wf.Plan(w.L, w.n_wave, w.n_hist, w.H, w.D).set_rope(w.F, w.gh, w.gw)
+    kc1 = torch.zeros((w.R, w.L, w.H, w.D), dtype=torch.bfloat16, device=dev)
+    vc1, kc2, vc2 = kc1.clone(), kc1.clone(), kc1.clone()
+    q_out = torch.empty_like(q)
+    wf.wf_qk_norm_rope_append(plan, 2, q, k, v, None, gq, gk, q_out, kc1, vc1)
+    q_inplace = q.clone()
+    wf.wf_qk_norm_rope_append(plan, 2, q_inplace, k, v, None, gq, gk, q_inplace, kc2, vc2)
+    torch.cuda.synchronize()
+    assert wf.wf_sync_status(plan) == wf.WF_OK
+    assert torch.equal(q_inplace.view(torch.int16), q_out.view(torch.int16))
+    assert torch.equal(kc1.view(torch.int16), kc2.view(torch.int16))
+    assert torch.equal(vc1.view(torch.int16), vc2.view(torch.int16))
+    plan.destroy()
