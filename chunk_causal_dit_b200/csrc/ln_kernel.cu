@@ -33,8 +33,11 @@ layer_norm_modulate_kernel(const uint16_t *__restrict__ x, const float *__restri
 {
     // shift and scale of the group of the block's first row, staged while the
     // row loads are in flight (a block's rows straddle two groups only at a
-    // chunk boundary; such rows read their own group's rows from global memory)
-    extern __shared__ float4 s_mod[];            // [C/4] shift, then [C/4] scale
+    // chunk boundary; such rows read their own group's rows from global memory).
+    // Staged de-interleaved: the first four floats of every 8-float piece, then
+    // the last four, so that a warp's 16-byte reads of one half are contiguous
+    // (interleaved, lanes 32 bytes apart would take twice the wavefronts).
+    extern __shared__ float4 s_mod[];            // shift lo, shift hi, scale lo, scale hi: [C/8] each
     const int lane = threadIdx.x & 31;
     const long row0 = static_cast<long>(blockIdx.x) * kRowsPerBlock;
     const long row = row0 + (threadIdx.x >> 5);
@@ -48,12 +51,14 @@ layer_norm_modulate_kernel(const uint16_t *__restrict__ x, const float *__restri
         w[i] = (live && j < pieces) ? __ldcs(src + j) : make_uint4(0u, 0u, 0u, 0u);
     }
     const long g0 = row0 / rows_per_group;
+    const int q = C / 8;                         // pieces per row
     {
         const float4 *sh = reinterpret_cast<const float4 *>(shift + g0 * C);
         const float4 *sc = reinterpret_cast<const float4 *>(scale + g0 * C);
         for (int i = threadIdx.x; i < C / 4; i += 32 * kRowsPerBlock) {
-            s_mod[i] = __ldg(sh + i);
-            s_mod[C / 4 + i] = __ldg(sc + i);
+            const int piece = i >> 1, half = i & 1;
+            s_mod[half * q + piece] = __ldg(sh + i);
+            s_mod[2 * q + half * q + piece] = __ldg(sc + i);
         }
     }
     __syncthreads();
@@ -85,16 +90,19 @@ layer_norm_modulate_kernel(const uint16_t *__restrict__ x, const float *__restri
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
     const float rstd = rsqrtf(v / static_cast<float>(C) + eps);
     const long g = row / rows_per_group;
-    const float4 *sh4 = g == g0 ? s_mod : reinterpret_cast<const float4 *>(shift + g * C);
-    const float4 *sc4 = g == g0 ? s_mod + C / 4 : reinterpret_cast<const float4 *>(scale + g * C);
+    const bool staged = g == g0;
+    const float4 *sh4 = reinterpret_cast<const float4 *>(shift + g * C);
+    const float4 *sc4 = reinterpret_cast<const float4 *>(scale + g * C);
     uint4 *dst = reinterpret_cast<uint4 *>(y + row * C);
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
         const int j = lane + 32 * i;
         if (j >= pieces) break;
         const uint32_t u[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
-        const float4 sa = sh4[2 * j], sb = sh4[2 * j + 1];
-        const float4 ca = sc4[2 * j], cb = sc4[2 * j + 1];
+        const float4 sa = staged ? s_mod[j] : __ldg(sh4 + 2 * j);
+        const float4 sb = staged ? s_mod[q + j] : __ldg(sh4 + 2 * j + 1);
+        const float4 ca = staged ? s_mod[2 * q + j] : __ldg(sc4 + 2 * j);
+        const float4 cb = staged ? s_mod[3 * q + j] : __ldg(sc4 + 2 * j + 1);
         const float shv[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
         const float scv[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
         uint32_t o[4];
