@@ -17,8 +17,9 @@
 // site, work counter) on its stream before the kernel runs, so calls whose work
 // overlaps on the GPU (different streams, no ordering between them) race on it
 // and must not be issued.  The kernel's timeout status is recorded in the block
-// but this entry point has no way to return it: use the plan API when the
-// status is needed.
+// but this entry point has no way to return it, so a call whose bounded wait
+// ran out (output partly written) cannot be told from a good one here: use the
+// plan API and wf_sync_status when the status is needed.
 #include <cudaTypedefs.h>
 
 #include <climits>
@@ -43,62 +44,60 @@ static_assert(sizeof(wf::DeviceWords) <= kNoAllocScratchBytes, "scratch block to
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 // Host code may not use g_noalloc_scratch as an address: on the host it names a
-// shadow variable, not device memory.  The device address is fetched once per
-// device, with that device current, and cached here.
+// shadow variable, not device memory.  The device address is looked up with
+// cudaGetSymbolAddress, with the device current, and cached per device together
+// with the CUDA context it belongs to.  A context that is torn down and created
+// again (cudaDeviceReset, say) loads the module afresh and the array may move,
+// so a call made in another context than the cached one looks the address up
+// again instead of using a stale pointer.
 constexpr int kMaxDevices = 64;
+struct ScratchEntry {
+    CUcontext ctx;
+    void *addr;
+};
 std::mutex g_scratch_mu;
-void *g_scratch_addr[kMaxDevices] = {};
+ScratchEntry g_scratch[kMaxDevices] = {};
 
-int scratch_for_current_device(int dev, void **out)
+PFN_cuCtxGetCurrent_v4000 ctx_get_current()
 {
-    if (dev < 0 || dev >= kMaxDevices) return WF_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (g_scratch_addr[dev] == nullptr) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
-            (void)cudaGetLastError();
-            return WF_ERR_CUDA;
-        }
-        g_scratch_addr[dev] = p;
-    }
-    *out = g_scratch_addr[dev];
-    return WF_OK;
-}
-
-PFN_cuTensorMapEncodeTiled_v12000 noalloc_map_encoder()
-{
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
     static std::once_flag once;
     std::call_once(once, [] {
         void *ptr = nullptr;
         cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) ==
                 cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+            fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(ptr);
         else
             (void)cudaGetLastError();
     });
     return fn;
 }
 
-// Same tensor maps as the plan API: (D, H, rows, chunk-or-slot), box 64x1x128x1,
-// 128-byte swizzle, rows past the extent read as zero.
-bool noalloc_map(CUtensorMap *map, const void *base, int D, int H, int L, int n3)
+int scratch_for_current_device(int dev, void **out)
 {
-    auto enc = noalloc_map_encoder();
-    if (!enc) return false;
-    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
-                                static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(n3)};
-    const cuuint64_t row = static_cast<cuuint64_t>(H) * D * 2;
-    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, row,
-                                   row * static_cast<cuuint64_t>(L)};
-    const cuuint32_t box[4] = {64, 1, 128, 1};
-    const cuuint32_t estr[4] = {1, 1, 1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
-               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    if (dev < 0 || dev >= kMaxDevices) return WF_ERR_UNSUPPORTED;
+    auto get_ctx = ctx_get_current();
+    if (get_ctx == nullptr) return WF_ERR_CUDA;
+    CUcontext ctx = nullptr;
+    if (get_ctx(&ctx) != CUDA_SUCCESS) return WF_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    ScratchEntry &e = g_scratch[dev];
+    if (ctx == nullptr || e.addr == nullptr || e.ctx != ctx) {
+        // the lookup also makes the device's primary context current when no
+        // context is yet, which is why the key is read again after it
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr ||
+            get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) {
+            (void)cudaGetLastError();
+            return WF_ERR_CUDA;
+        }
+        e.ctx = ctx;
+        e.addr = p;
+    }
+    *out = e.addr;
+    return WF_OK;
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -111,19 +110,15 @@ extern "C" int wf_chunk_causal_attn_noalloc(int chunk_tokens, int n_wave_chunks,
                                             const void *v_cache, void *o, float *lse,
                                             void *stream)
 {
+    wf::NvtxRange nvtx_range("wf_chunk_causal_attn_noalloc");
     // the plan API's shape rules
-    if (chunk_tokens < 1 || n_wave_chunks < 1 || n_hist_chunks < 0 || heads < 1 || round < 0)
-        return WF_ERR_INVALID_ARG;
-    if (head_dim != 64 && head_dim != 128) return WF_ERR_UNSUPPORTED;
+    if (round < 0) return WF_ERR_INVALID_ARG;
+    if (int st = wf::check_round_shape(chunk_tokens, n_wave_chunks, n_hist_chunks, heads, head_dim))
+        return st;
     const long long T = static_cast<long long>(chunk_tokens) * n_wave_chunks;
     const long long R = static_cast<long long>(n_hist_chunks) + n_wave_chunks;
-    const long long hd = static_cast<long long>(heads) * head_dim;
-    if (T * hd >= (1ll << 31) || R * chunk_tokens * hd >= (1ll << 40) || R > INT_MAX)
-        return WF_ERR_INVALID_ARG;
     const int n_ktiles = (chunk_tokens + 127) / 128;
     const int n_qpairs = (n_ktiles + 1) / 2;
-    if (static_cast<long long>(heads) * n_wave_chunks * n_qpairs >= INT_MAX)
-        return WF_ERR_INVALID_ARG;
     if (!q_out || !k_cache || !v_cache || !o) return WF_ERR_INVALID_ARG;
     if (!aligned16(q_out) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
         (reinterpret_cast<uintptr_t>(lse) & 3u))
@@ -142,9 +137,11 @@ extern "C" int wf_chunk_causal_attn_noalloc(int chunk_tokens, int n_wave_chunks,
     if (int s = scratch_for_current_device(dev, &scratch)) return s;
 
     CUtensorMap mq, mk, mv;
-    if (!noalloc_map(&mq, q_out, head_dim, heads, chunk_tokens, n_wave_chunks) ||
-        !noalloc_map(&mk, k_cache, head_dim, heads, chunk_tokens, static_cast<int>(R)) ||
-        !noalloc_map(&mv, v_cache, head_dim, heads, chunk_tokens, static_cast<int>(R)))
+    if (!wf::encode_map(&mq, q_out, head_dim, heads, chunk_tokens, chunk_tokens, n_wave_chunks) ||
+        !wf::encode_map(&mk, k_cache, head_dim, heads, chunk_tokens, chunk_tokens,
+                        static_cast<int>(R)) ||
+        !wf::encode_map(&mv, v_cache, head_dim, heads, chunk_tokens, chunk_tokens,
+                        static_cast<int>(R)))
         return WF_ERR_CUDA;
 
     wf::AttnParams a;

@@ -34,22 +34,7 @@ cudaError_t launch_layer_norm_modulate(const uint16_t *x, const float *shift, co
 int ln_max_channels();
 }  // namespace wf
 
-namespace {
-
-constexpr unsigned long long kDefaultWaitLimit = 1ull << 32;   // ~2 s of SM clock
-
-bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-void fill_rope_table(wf::RopeParams &r, double theta)
-{
-    const int width[3] = {r.dt, r.dh, r.dw};
-    int pair = 0;
-    for (int a = 0; a < 3; ++a)
-        for (int i = 0; i < width[a] / 2; ++i, ++pair) {
-            r.omega[pair] = std::pow(theta, -2.0 * i / width[a]);
-            r.axis[pair] = static_cast<int8_t>(a);
-        }
-}
+namespace wf {
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 {
@@ -71,7 +56,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 // 4-D map over a [n3][n2][H][D] bf16 tensor (slot/chunk, row, head, channel),
 // box = 64 channels x 1 head x box_rows rows x 1 slot, 128-byte swizzle, OOB rows read 0.
 bool encode_map(CUtensorMap *map, const void *base, int D, int H, int n2, int n2_stride_rows,
-                int n3, int box_rows = 128)
+                int n3, int box_rows)
 {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
@@ -89,11 +74,50 @@ bool encode_map(CUtensorMap *map, const void *base, int D, int H, int n2, int n2
     return r == CUDA_SUCCESS;
 }
 
+// The shape rules of a wave round (wf_plan and the plan-free attention entry
+// point apply the same ones): positive sizes, head_dim 64 or 128, and index
+// ranges that fit the kernels' int / 40-bit arithmetic.
+int check_round_shape(int chunk_tokens, int n_wave_chunks, int n_hist_chunks, int heads,
+                      int head_dim)
+{
+    if (chunk_tokens < 1 || n_wave_chunks < 1 || n_hist_chunks < 0 || heads < 1)
+        return WF_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return WF_ERR_UNSUPPORTED;
+    const long long T = static_cast<long long>(chunk_tokens) * n_wave_chunks;
+    const long long R = static_cast<long long>(n_hist_chunks) + n_wave_chunks;
+    const long long hd = static_cast<long long>(heads) * head_dim;
+    if (T * hd >= (1ll << 31) || R * chunk_tokens * hd >= (1ll << 40) || R > INT_MAX)
+        return WF_ERR_INVALID_ARG;
+    const long long qtiles = (chunk_tokens + 127) / 128;
+    if (static_cast<long long>(heads) * n_wave_chunks * ((qtiles + 1) / 2) >= INT_MAX)
+        return WF_ERR_INVALID_ARG;
+    return WF_OK;
+}
+
+}  // namespace wf
+
+namespace {
+
+constexpr unsigned long long kDefaultWaitLimit = 1ull << 32;   // ~2 s of SM clock
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+void fill_rope_table(wf::RopeParams &r, double theta)
+{
+    const int width[3] = {r.dt, r.dh, r.dw};
+    int pair = 0;
+    for (int a = 0; a < 3; ++a)
+        for (int i = 0; i < width[a] / 2; ++i, ++pair) {
+            r.omega[pair] = std::pow(theta, -2.0 * i / width[a]);
+            r.axis[pair] = static_cast<int8_t>(a);
+        }
+}
+
 // The same map over a [n3][n2][H][D] array of one-byte E4M3 codes: box = D bytes
 // (one 128-byte swizzle row at D = 128) x 1 head x 128 rows x 1.
 bool encode_map_u8(CUtensorMap *map, const void *base, int D, int H, int n2, int n3)
 {
-    auto enc = tensor_map_encoder();
+    auto enc = wf::tensor_map_encoder();
     if (!enc) return false;
     const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
                                 static_cast<cuuint64_t>(n2), static_cast<cuuint64_t>(n3)};
@@ -115,7 +139,7 @@ bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0
 // innermost): box = 64 columns x 128 rows, 128-byte swizzle, out-of-range reads 0.
 bool encode_map_2d(CUtensorMap *map, const void *base, long rows, long cols)
 {
-    auto enc = tensor_map_encoder();
+    auto enc = wf::tensor_map_encoder();
     if (!enc) return false;
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
@@ -157,17 +181,9 @@ int wf_plan(int chunk_tokens, int n_wave_chunks, int n_hist_chunks, int heads, i
 {
     if (out == nullptr) return WF_ERR_INVALID_ARG;
     *out = nullptr;
-    if (chunk_tokens < 1 || n_wave_chunks < 1 || n_hist_chunks < 0 || heads < 1)
-        return WF_ERR_INVALID_ARG;
-    if (head_dim != 64 && head_dim != 128) return WF_ERR_UNSUPPORTED;
-    const long long T = static_cast<long long>(chunk_tokens) * n_wave_chunks;
+    if (int st = wf::check_round_shape(chunk_tokens, n_wave_chunks, n_hist_chunks, heads, head_dim))
+        return st;
     const long long R = static_cast<long long>(n_hist_chunks) + n_wave_chunks;
-    const long long hd = static_cast<long long>(heads) * head_dim;
-    if (T * hd >= (1ll << 31) || R * chunk_tokens * hd >= (1ll << 40) || R > INT_MAX)
-        return WF_ERR_INVALID_ARG;
-    const long long qtiles = (chunk_tokens + 127) / 128;
-    if (static_cast<long long>(heads) * n_wave_chunks * ((qtiles + 1) / 2) >= INT_MAX)
-        return WF_ERR_INVALID_ARG;
 
     wf_plan_s *p = new (std::nothrow) wf_plan_s();
     if (p == nullptr) return WF_ERR_CUDA;
@@ -303,6 +319,7 @@ int wf_qk_norm_rope_append(wf_plan_t p, long round, const void *q, const void *k
                            const int32_t *pos_thw, const float *gamma_q, const float *gamma_k,
                            void *q_out, void *k_cache, void *v_cache, void *stream)
 {
+    wf::NvtxRange nvtx_range("wf_qk_norm_rope_append");
     if (p == nullptr || round < 0) return WF_ERR_INVALID_ARG;
     if (!q || !k || !v || !gamma_q || !gamma_k || !q_out || !k_cache || !v_cache)
         return WF_ERR_INVALID_ARG;
@@ -340,6 +357,7 @@ int wf_qk_norm_rope_append(wf_plan_t p, long round, const void *q, const void *k
 int wf_chunk_causal_attn(wf_plan_t p, long round, const void *q_out, const void *k_cache,
                          const void *v_cache, void *o, float *lse, void *stream)
 {
+    wf::NvtxRange nvtx_range("wf_chunk_causal_attn");
     if (p == nullptr || round < 0) return WF_ERR_INVALID_ARG;
     if (!q_out || !k_cache || !v_cache || !o) return WF_ERR_INVALID_ARG;
     if (!aligned16(q_out) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
@@ -348,9 +366,9 @@ int wf_chunk_causal_attn(wf_plan_t p, long round, const void *q_out, const void 
     if (int s = check_device(p)) return s;
 
     CUtensorMap mq, mk, mv;
-    if (!encode_map(&mq, q_out, p->D, p->H, p->L, p->L, p->W) ||
-        !encode_map(&mk, k_cache, p->D, p->H, p->L, p->L, p->R) ||
-        !encode_map(&mv, v_cache, p->D, p->H, p->L, p->L, p->R))
+    if (!wf::encode_map(&mq, q_out, p->D, p->H, p->L, p->L, p->W) ||
+        !wf::encode_map(&mk, k_cache, p->D, p->H, p->L, p->L, p->R) ||
+        !wf::encode_map(&mv, v_cache, p->D, p->H, p->L, p->L, p->R))
         return WF_ERR_CUDA;
 
     wf::AttnParams a;
@@ -376,7 +394,7 @@ int wf_chunk_causal_attn(wf_plan_t p, long round, const void *q_out, const void 
     cudaError_t e;
     if (pair) {
         CUtensorMap mk64;
-        if (!encode_map(&mk64, k_cache, p->D, p->H, p->L, p->L, p->R, 64)) return WF_ERR_CUDA;
+        if (!wf::encode_map(&mk64, k_cache, p->D, p->H, p->L, p->L, p->R, 64)) return WF_ERR_CUDA;
         e = wf::launch_attn_pair(mq, mk64, mv, a, static_cast<cudaStream_t>(stream));
     } else {
         const int grid = a.n_units < p->num_sms ? a.n_units : p->num_sms;
@@ -387,6 +405,7 @@ int wf_chunk_causal_attn(wf_plan_t p, long round, const void *q_out, const void 
 
 int wf_quantize_q_fp8(wf_plan_t p, const void *q_out, void *q8, float *q_scale, void *stream)
 {
+    wf::NvtxRange nvtx_range("wf_quantize_q_fp8");
     if (p == nullptr || !q_out || !q8 || !q_scale) return WF_ERR_INVALID_ARG;
     if (!aligned16(q_out) || !aligned16(q8) || !aligned4(q_scale)) return WF_ERR_INVALID_ARG;
     if (int s = check_device(p)) return s;
@@ -400,6 +419,7 @@ int wf_quantize_q_fp8(wf_plan_t p, const void *q_out, void *q8, float *q_scale, 
 int wf_quantize_k_fp8(wf_plan_t p, long first_chunk, int n_chunks, const void *k_cache,
                       void *k8_cache, float *k_scale, void *stream)
 {
+    wf::NvtxRange nvtx_range("wf_quantize_k_fp8");
     if (p == nullptr || first_chunk < 0 || n_chunks < 0 || n_chunks > p->R) return WF_ERR_INVALID_ARG;
     if (!k_cache || !k8_cache || !k_scale) return WF_ERR_INVALID_ARG;
     if (!aligned16(k_cache) || !aligned16(k8_cache) || !aligned4(k_scale)) return WF_ERR_INVALID_ARG;
@@ -415,6 +435,7 @@ int wf_chunk_causal_attn_fp8qk(wf_plan_t p, long round, const void *q8, const fl
                                const void *k8_cache, const float *k_scale, const void *v_cache,
                                void *o, float *lse, void *stream)
 {
+    wf::NvtxRange nvtx_range("wf_chunk_causal_attn_fp8qk");
     if (p == nullptr || round < 0) return WF_ERR_INVALID_ARG;
     if (p->D != 128) return WF_ERR_UNSUPPORTED;
     if (!q8 || !q_scale || !k8_cache || !k_scale || !v_cache || !o) return WF_ERR_INVALID_ARG;
@@ -426,7 +447,7 @@ int wf_chunk_causal_attn_fp8qk(wf_plan_t p, long round, const void *q8, const fl
     CUtensorMap mq, mk, mv;
     if (!encode_map_u8(&mq, q8, p->D, p->H, p->L, p->W) ||
         !encode_map_u8(&mk, k8_cache, p->D, p->H, p->L, p->R) ||
-        !encode_map(&mv, v_cache, p->D, p->H, p->L, p->L, p->R))
+        !wf::encode_map(&mv, v_cache, p->D, p->H, p->L, p->L, p->R))
         return WF_ERR_CUDA;
 
     wf::AttnParams a;
@@ -457,6 +478,7 @@ int wf_linear(wf_plan_t p, int M, int N, int K, const void *x, const void *w, co
               int epilogue, const float *gate, const void *resid, int rows_per_group, void *y,
               void *stream)
 {
+    wf::NvtxRange nvtx_range("wf_linear");
     if (p == nullptr || M < 0 || N < 32 || K < 8 || N % 32 || K % 8) return WF_ERR_INVALID_ARG;
     if (epilogue < WF_EPI_STORE || epilogue > WF_EPI_GATED_RESIDUAL) return WF_ERR_INVALID_ARG;
     if (M == 0) return WF_OK;                        // nothing to compute, nothing is read
@@ -491,6 +513,7 @@ int wf_qkv_proj_norm_rope_append(wf_plan_t p, long round, int hidden, const void
                                  const float *gamma_k, void *q_out, void *k_cache, void *v_cache,
                                  void *stream)
 {
+    wf::NvtxRange nvtx_range("wf_qkv_proj_norm_rope_append");
     if (p == nullptr || round < 0 || hidden < 8 || hidden % 8) return WF_ERR_INVALID_ARG;
     if (!x || !w_qkv || !gamma_q || !gamma_k || !q_out || !k_cache || !v_cache)
         return WF_ERR_INVALID_ARG;
@@ -541,6 +564,7 @@ int wf_qkv_proj_norm_rope_append(wf_plan_t p, long round, int hidden, const void
 int wf_layer_norm_modulate(wf_plan_t p, int M, int C, const void *x, const float *shift,
                            const float *scale, int rows_per_group, void *y, void *stream)
 {
+    wf::NvtxRange nvtx_range("wf_layer_norm_modulate");
     if (p == nullptr || M < 0 || C < 8 || C % 8 || rows_per_group < 1) return WF_ERR_INVALID_ARG;
     if (C > wf::ln_max_channels()) return WF_ERR_UNSUPPORTED;
     if (!x || !shift || !scale || !y || !aligned16(x) || !aligned16(shift) || !aligned16(scale) ||

@@ -5,6 +5,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #ifdef __CUDACC__
 #define WF_HD __host__ __device__ __forceinline__
@@ -113,6 +114,26 @@ struct GemmParams {
     int withhold;             // test hook: no CTA issues (or arms) its first stage's copies
     DeviceWords *words;
 };
+
+// NVTX range around a host call of the C ABI (header-only NVTX v3: without a
+// profiler attached a push/pop is a null-callback check), so that a timeline
+// shows each launch under the library call that made it.
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
+
+// Host helpers shared by the plan API and the plan-free attention entry point
+// (defined in wf_api.cu).
+// 4-D TMA map over a [n3][n2][H][D] bf16 tensor, box 64 x 1 x box_rows x 1,
+// 128-byte swizzle, rows past n2 read as zero.
+bool encode_map(CUtensorMap *map, const void *base, int D, int H, int n2, int n2_stride_rows,
+                int n3, int box_rows = 128);
+// WF_OK, or the status wf_plan returns for this shape.
+int check_round_shape(int chunk_tokens, int n_wave_chunks, int n_hist_chunks, int heads,
+                      int head_dim);
 
 }  // namespace wf
 

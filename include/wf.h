@@ -66,6 +66,10 @@ typedef enum wf_status {
 typedef struct wf_plan_s *wf_plan_t;
 
 /* Build a plan for one layer's wave round.
+ * Passage: "Wave Forcing" abstract -- a wave is S chunks at staggered denoising
+ * steps plus one cache-refresh chunk (W = S + 1), with a rolling history; the
+ * airadar.tv summary, usage section, gives the sizes (--rf-step 4 --wp-size 5:
+ * W = 5; 3-latent-frame chunks).
  * chunk_tokens L >= 1, n_wave_chunks W >= 1, n_hist_chunks Hh >= 0, heads H >= 1,
  * head_dim D in {64, 128}; T*H*D must fit in 2^31 elements per tensor.
  * Host work only, plus a 256-byte device allocation (status word and the
@@ -128,10 +132,17 @@ WF_API void wf_plan_destroy(wf_plan_t plan);
 WF_API size_t wf_cache_bytes(wf_plan_t plan);
 
 /* Useful attention FLOPs of round r: 4*H*D*L^2 * sum_c (min(Hh, r) + c + 1),
+ * counting the key chunks that chunk-wise causal attention ("Wave Forcing"
+ * abstract) lets wave chunk c see: the valid history plus wave chunks 0..c;
  * i.e. QK^T and PV over visible, unpadded pairs.  -1 for a NULL plan. */
 WF_API double wf_useful_flops(wf_plan_t plan, long round);
 
 /* Fused per-head RMSNorm(q, k) * gamma, 3D RoPE, and ring append.
+ * Passage: "Wave Forcing" abstract and the airadar.tv summary's mechanism
+ * paragraph -- each layer's K/V is handed to the later chunks early (Wave
+ * Parallelism); on one GPU that hand-over is this write into the ring the
+ * attention reads.  The per-head norm and (t,h,w) RoPE are those of the Wan2.1
+ * DiT the pages run (their formulas are not printed; plain definitions here).
  * For every wave token n (chunk c = n / L) and head h:
  *   q_out[n,h] = bf16(RoPE(pos[n], RMSNorm(q[n,h]) * gamma_q[h]))
  *   k_cache[(r+c) mod R, n mod L, h] = bf16(RoPE(pos[n], RMSNorm(k[n,h]) * gamma_k[h]))
@@ -147,7 +158,11 @@ WF_API int wf_qk_norm_rope_append(wf_plan_t plan, long round,
                            void *q_out, void *k_cache, void *v_cache,
                            void *stream);
 
-/* Chunk-causal attention of round r.  For query token n of wave chunk c, head h:
+/* Chunk-causal attention of round r.
+ * Passage: "Wave Forcing" abstract -- chunk-wise causal attention: a chunk attends
+ * to the history cache and to the earlier (cleaner) chunks of the wave even while
+ * those are still being denoised, and bidirectionally inside itself.
+ * For query token n of wave chunk c, head h:
  *   O[n,h] = softmax_j(q_out[n,h] . K_j / sqrt(D)) V_j
  * over every token j of the min(Hh, r) history chunks and of wave chunks 0..c
  * (bidirectional inside a chunk), read from the ring slots written by
@@ -282,12 +297,14 @@ WF_API const char *wf_status_string(int status);
  * device block the kernel's scratch (status word, timeout site, work counter)
  * lives in a 256-byte block compiled into the library, present on every GPU
  * that loads it until the process exits; no cudaMalloc, cudaFree or
- * allocating library call is made.  The first call on a device looks up that
- * block's device address (cudaGetSymbolAddress); make that first call before
- * any stream capture.  All calls on a device share the block: each clears what
- * must start at zero on its own stream, and calls that overlap on the GPU race
- * on it.  A device-side timeout is recorded in the block but not reported
- * here.  Returns WF_OK, WF_ERR_INVALID_ARG / WF_ERR_UNSUPPORTED for shapes or
+ * allocating library call is made.  The first call on a device (and the first
+ * after that device's context was created again, e.g. after cudaDeviceReset)
+ * looks up that block's device address (cudaGetSymbolAddress); make that first
+ * call before any stream capture.  All calls on a device share the block: each
+ * clears what must start at zero on its own stream, and calls that overlap on
+ * the GPU race on it.  A device-side timeout is recorded in the block but not
+ * reported here: such a call still returns WF_OK with o partly written, so a
+ * caller that needs the status must use the plan API and wf_sync_status.  Returns WF_OK, WF_ERR_INVALID_ARG / WF_ERR_UNSUPPORTED for shapes or
  * pointers the plan API would reject, WF_ERR_NO_DEVICE, WF_ERR_DEVICE or
  * WF_ERR_CUDA. */
 WF_API int wf_chunk_causal_attn_noalloc(int chunk_tokens, int n_wave_chunks, int n_hist_chunks,

@@ -13,8 +13,8 @@ import torch
 import oracle
 from chunk_causal_dit_b200 import build as wf_build
 from chunk_causal_dit_b200 import inputs as wi
-from tests.wfcase import (assert_attention_close, assert_attention_within_rounding,
-                          rand_bf16, sample_rows)
+from tests.wfcase import (assert_attention_close, assert_attention_close_scaled,
+                          assert_attention_within_rounding, rand_bf16, sample_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -160,11 +160,11 @@ def test_score_jump_far_above_the_running_reference(wf, D, kernel):
         hit[n * H + h] = True
     # The big keys also pull rows that merely correlate with the targeted
     # queries towards a single V row, so |O| reaches ~4.5 where one bf16
-    # rounding alone exceeds the 1e-2 max-abs bar: every row is held to the
-    # elementwise rounding bound, and all rows together to the mean bar.
+    # rounding alone exceeds the 1e-2 max-abs bar: elements with |O| > 1 are
+    # held to the elementwise rounding bound, the rest to the 1e-2 bar, and
+    # all together to the mean bar.
     v_absmax = float(vc.float().abs().max())
-    assert_attention_within_rounding(got, ref, v_absmax, "score jump D=%d" % D)
-    assert float(np.abs(got - ref).mean()) <= 1e-3
+    assert_attention_close_scaled(got, ref, v_absmax, "score jump D=%d" % D)
     for n, h, key in targets:
         v = vc[key[0], key[1], h].float().cpu().numpy()
         assert np.max(np.abs(o[n, h].float().cpu().numpy() - v)) <= 2.0 ** -6 * np.abs(v).max()
