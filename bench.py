@@ -242,8 +242,9 @@ def run_ours(args, rank, world, local):
     r0 = w.n_hist
     flops_step = wf.wf_useful_flops(plan, r0)
     tensor_bytes = w.T * w.H * w.D * 2
-    append_bytes = 12 * w.T * w.H * w.D
     fp8 = args.attn == "fp8qk"
+    # bf16: read q, k, v, write q', K', V; fused FP8: the q' write is one code byte
+    append_bytes = (11 if fp8 else 12) * w.T * w.H * w.D
     if fp8:
         # E4M3 copies of q_out (per row) and of the key ring (per 128-row tile);
         # the history chunks were quantized when they were appended
@@ -254,17 +255,16 @@ def run_ours(args, rank, world, local):
         k_scale = torch.empty((w.R, nt, w.H), dtype=torch.float32, device=dev)
         wf.wf_quantize_k_fp8(plan, 0, w.n_hist, kc, k8, k_scale, stream)
 
-    def attention(r):
+    def step(r):
         if fp8:
-            wf.wf_quantize_q_fp8(plan, q_out, q8, q_scale, stream)
+            # the append writes q's E4M3 codes; the wave's K chunks are quantized after it
+            wf.wf_qk_norm_rope_append_fp8q(plan, r, q, k, v, None, gq, gk, None, q8, q_scale,
+                                           kc, vc, stream)
             wf.wf_quantize_k_fp8(plan, r, w.n_wave, kc, k8, k_scale, stream)
             wf.wf_chunk_causal_attn_fp8qk(plan, r, q8, q_scale, k8, k_scale, vc, o, None, stream)
         else:
+            wf.wf_qk_norm_rope_append(plan, r, q, k, v, None, gq, gk, q_out, kc, vc, stream)
             wf.wf_chunk_causal_attn(plan, r, q_out, kc, vc, o, None, stream)
-
-    def step(r):
-        wf.wf_qk_norm_rope_append(plan, r, q, k, v, None, gq, gk, q_out, kc, vc, stream)
-        attention(r)
 
     rnd = r0
     for _ in range(args.warmup):
@@ -288,10 +288,13 @@ def run_ours(args, rank, world, local):
     for i in range(args.steps):
         e0, e1, eq, e2 = ev[i]
         e0.record(stream)
-        wf.wf_qk_norm_rope_append(plan, rnd, q, k, v, None, gq, gk, q_out, kc, vc, stream)
+        if fp8:
+            wf.wf_qk_norm_rope_append_fp8q(plan, rnd, q, k, v, None, gq, gk, None, q8, q_scale,
+                                           kc, vc, stream)
+        else:
+            wf.wf_qk_norm_rope_append(plan, rnd, q, k, v, None, gq, gk, q_out, kc, vc, stream)
         e1.record(stream)
         if fp8:
-            wf.wf_quantize_q_fp8(plan, q_out, q8, q_scale, stream)
             wf.wf_quantize_k_fp8(plan, rnd, w.n_wave, kc, k8, k_scale, stream)
             eq.record(stream)
             wf.wf_chunk_causal_attn_fp8qk(plan, rnd, q8, q_scale, k8, k_scale, vc, o, None,
@@ -417,7 +420,7 @@ def run_ours(args, rank, world, local):
             "useful_flop_per_launch": flops_step,
         },
         "append": {
-            "kernel": "qk_norm_rope_append_kernel",
+            "kernel": "qk_norm_rope_append_kernel" + ("<128, q8>" if fp8 else ""),
             "bound": "hbm",
             "ms_per_launch": round(append_ms, 5),
             "achieved": round(append_gbs, 1),
@@ -428,14 +431,15 @@ def run_ours(args, rank, world, local):
             "bytes_per_launch": append_bytes,
         },
         **({"quantize": {
-            "kernels": "quantize_rows_kernel + quantize_tiles_kernel (wave chunks)",
+            "kernels": "quantize_tiles_kernel (the wave's key chunks; q is quantized in the "
+                       "append)",
             "bound": "hbm",
             "ms_per_step": round(quant_ms, 5),
-            "achieved": round(6 * w.T * w.H * w.D / (quant_ms * 1e-3) / 1e9, 1),
+            "achieved": round(3 * w.T * w.H * w.D / (quant_ms * 1e-3) / 1e9, 1),
             "peak": hbm,
             "unit": "GB/s",
-            "frac": round(6 * w.T * w.H * w.D / (quant_ms * 1e-3) / 1e9 / hbm, 4),
-            "bytes_per_step": 6 * w.T * w.H * w.D,
+            "frac": round(3 * w.T * w.H * w.D / (quant_ms * 1e-3) / 1e9 / hbm, 4),
+            "bytes_per_step": 3 * w.T * w.H * w.D,
         }} if fp8 else {}),
         "e2e": {
             "value": round(aggregate_tflops(world, flops_step, e2e_ms), 3),
@@ -444,7 +448,7 @@ def run_ours(args, rank, world, local):
             "h2d_bytes_per_step": 3 * tensor_bytes,
             "d2h_bytes_per_step": tensor_bytes,
         },
-        "gpu_launches": (5 if fp8 else 2) * args.steps,
+        "gpu_launches": (3 if fp8 else 2) * args.steps,
         "clocks": clk,
     }
     if block is not None:
@@ -492,11 +496,14 @@ def measure_single_layer(w, steps, warmup, dev, peaks, fp8=False, seed=0):
     def step(r, e=None):
         if e is not None:
             e[0].record(stream)
-        wf.wf_qk_norm_rope_append(plan, r, q, k, v, None, gq, gk, q_out, kc, vc, stream)
+        if fp8:
+            wf.wf_qk_norm_rope_append_fp8q(plan, r, q, k, v, None, gq, gk, None, q8, q_scale,
+                                           kc, vc, stream)
+        else:
+            wf.wf_qk_norm_rope_append(plan, r, q, k, v, None, gq, gk, q_out, kc, vc, stream)
         if e is not None:
             e[1].record(stream)
         if fp8:
-            wf.wf_quantize_q_fp8(plan, q_out, q8, q_scale, stream)
             wf.wf_quantize_k_fp8(plan, r, w.n_wave, kc, k8, k_scale, stream)
         if e is not None:
             e[2].record(stream)
@@ -534,7 +541,7 @@ def measure_single_layer(w, steps, warmup, dev, peaks, fp8=False, seed=0):
     stp = statistics.mean(e[0].elapsed_time(e[3]) for e in ev)
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     peak_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * (4.0 / 3.0 if fp8 else 1.0)
-    append_bytes = 12 * w.T * w.H * w.D
+    append_bytes = (11 if fp8 else 12) * w.T * w.H * w.D
     d = {"workload": w.name, "heads": w.H, "head_dim": w.D, "chunk_tokens": w.L,
          "wave_chunks": w.n_wave, "history_chunks": w.n_hist, "steps": steps, "warmup": warmup,
          "attention_ms": round(att, 5), "append_us": round(1e3 * app, 2),
@@ -551,7 +558,7 @@ def measure_single_layer(w, steps, warmup, dev, peaks, fp8=False, seed=0):
     else:
         d["note"] = "latency only: the working set fits in L2, no roofline claim"
     if fp8:
-        qbytes = 6 * w.T * w.H * w.D
+        qbytes = 3 * w.T * w.H * w.D           # the wave's key chunks (q: in the append)
         d.update({"quantize_us": round(1e3 * qnt, 2),
                   "quantize_gbs": round(qbytes / (qnt * 1e-3) / 1e9, 1),
                   "quantize_frac": round(qbytes / (qnt * 1e-3) / 1e9 / hbm, 4),

@@ -16,8 +16,15 @@
 // pos * omega in fp64, reduced to [-pi, pi] in fp64, then fp32 sincos -- so the
 // fp32 error of the rotation stays a few ulps of the pair's length at any
 // position.
+//
+// The Q8 instantiation also quantizes each (token, head) row of q' to E4M3 for
+// the FP8 Q.K^T attention, in registers: the row's D / 8 threads reduce the
+// amax of the bf16-rounded q' with the same shuffles as the norm, then write
+// the codes and the row's scale (the rule of fp8_rule.cuh, so the bits equal
+// the stand-alone row quantizer's on q_out).  q_out itself is then optional.
 #include <cuda_bf16.h>
 
+#include "fp8_rule.cuh"
 #include "sm100.cuh"
 #include "wf_check.cuh"
 #include "wf_internal.h"
@@ -49,7 +56,7 @@ __device__ __forceinline__ uint4 pack8(const float (&y)[8])
     return u;
 }
 
-template <int D>
+template <int D, bool Q8>
 __global__ void __launch_bounds__(kMaxThreads) qk_norm_rope_append_kernel(const AppendParams p,
                                                                           DeviceWords *words)
 {
@@ -158,10 +165,24 @@ __global__ void __launch_bounds__(kMaxThreads) qk_norm_rope_append_kernel(const 
             yk[2 * e] = k0 * cs.x - k1 * cs.y;
             yk[2 * e + 1] = k0 * cs.y + k1 * cs.x;
         }
+        const uint4 q16 = pack8(yq);
+        float inv = 1.0f, qs = 1.0f;
+        if constexpr (Q8) {
+            // amax of the row's bf16 q' over its D / 8 threads (inactive lanes hold 0)
+            float a = absmax8(q16);
+#pragma unroll
+            for (int o = TPR / 2; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+            inv = fp8_inv(a);
+            qs = fp8_scale(a);
+        }
         if (active && WF_CHECKED(s_off[tl] >= 0)) {
             const long off = (n * p.H + h) * D + part * 8;
             const long coff = s_off[tl] + static_cast<long>(h) * D + part * 8;
-            *reinterpret_cast<uint4 *>(p.q_out + off) = pack8(yq);
+            if (!Q8 || p.q_out != nullptr) *reinterpret_cast<uint4 *>(p.q_out + off) = q16;
+            if constexpr (Q8) {
+                *reinterpret_cast<uint2 *>(p.q8 + off) = quant8(q16, inv);
+                if (part == 0) p.q_scale[static_cast<long>(h) * T + n] = qs;
+            }
             *reinterpret_cast<uint4 *>(p.k_cache + coff) = pack8(yk);
             *reinterpret_cast<uint4 *>(p.v_cache + coff) = uv[tl];
         }
@@ -182,10 +203,14 @@ cudaError_t launch_append(const AppendParams &p_in, int D, cudaStream_t stream, 
     const int by = (p.H + p.heads_per_block - 1) / p.heads_per_block;
     if (bx <= 0) return cudaSuccess;
     const dim3 grid(static_cast<unsigned>(bx), static_cast<unsigned>(by));
-    if (D == 128)
-        qk_norm_rope_append_kernel<128><<<grid, threads, 0, stream>>>(p, words);
-    else
-        qk_norm_rope_append_kernel<64><<<grid, threads, 0, stream>>>(p, words);
+    const bool q8 = p.q8 != nullptr;
+    if (D == 128) {
+        if (q8) qk_norm_rope_append_kernel<128, true><<<grid, threads, 0, stream>>>(p, words);
+        else qk_norm_rope_append_kernel<128, false><<<grid, threads, 0, stream>>>(p, words);
+    } else {
+        if (q8) qk_norm_rope_append_kernel<64, true><<<grid, threads, 0, stream>>>(p, words);
+        else qk_norm_rope_append_kernel<64, false><<<grid, threads, 0, stream>>>(p, words);
+    }
     return cudaGetLastError();
 }
 

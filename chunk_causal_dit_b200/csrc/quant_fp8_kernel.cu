@@ -7,51 +7,19 @@
 // W8A8 backends): scores come from 8-bit operands with per-block fp32 scales,
 // while P.V stays in bf16.
 //
-// Rule (exact, bit-for-bit what the oracle computes): for a group of values x
-// (a row for Q, a key tile for K), amax = max |x| (exact in fp32); the
-// dequantization scale is amax / 448 and the quantization multiplier 448 / amax,
-// both IEEE fp32 divisions (1 when amax = 0); code = E4M3 rounding, ties to
-// even, with saturation, of the IEEE fp32 product x * (448 / amax).
+// Rule (exact, bit-for-bit what the oracle computes): fp8_rule.cuh, applied to
+// a row for Q and to a 128-row key tile of one head for K.
 //
 // Both kernels are HBM-bound: 2 bytes read and 1 byte written per element.
 #include <cuda_bf16.h>
 
+#include "fp8_rule.cuh"
 #include "wf_check.cuh"
 #include "wf_internal.h"
 
 namespace wf {
 
 namespace {
-
-constexpr float kE4M3Max = 448.0f;
-
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-// two E4M3 codes in the low 16 bits: `lo` in bits 0-7, `hi` in bits 8-15
-__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi)
-{
-    uint16_t r;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-    return r;
-}
-
-__device__ __forceinline__ float fp8_scale(float amax)
-{
-    return amax > 0.0f ? __fdiv_rn(amax, kE4M3Max) : 1.0f;
-}
-
-__device__ __forceinline__ float fp8_inv(float amax)
-{
-    return amax > 0.0f ? __fdiv_rn(kE4M3Max, amax) : 1.0f;
-}
-
-// 4 codes of x0..x3 * inv, packed little-endian
-__device__ __forceinline__ uint32_t quant4(float x0, float x1, float x2, float x3, float inv)
-{
-    return e4m3x2(__fmul_rn(x0, inv), __fmul_rn(x1, inv)) |
-           (e4m3x2(__fmul_rn(x2, inv), __fmul_rn(x3, inv)) << 16);
-}
 
 __device__ __forceinline__ float warp_max(float v)
 {

@@ -315,16 +315,19 @@ double wf_useful_flops(wf_plan_t p, long round)
     return 4.0 * p->H * p->D * static_cast<double>(p->L) * p->L * chunks;
 }
 
-int wf_qk_norm_rope_append(wf_plan_t p, long round, const void *q, const void *k, const void *v,
-                           const int32_t *pos_thw, const float *gamma_q, const float *gamma_k,
-                           void *q_out, void *k_cache, void *v_cache, void *stream)
+// The append of both entry points below (q8 == nullptr: the plain append).
+static int append_common(wf_plan_t p, long round, const void *q, const void *k, const void *v,
+                         const int32_t *pos_thw, const float *gamma_q, const float *gamma_k,
+                         void *q_out, uint8_t *q8, float *q_scale, void *k_cache, void *v_cache,
+                         void *stream)
 {
-    wf::NvtxRange nvtx_range("wf_qk_norm_rope_append");
     if (p == nullptr || round < 0) return WF_ERR_INVALID_ARG;
-    if (!q || !k || !v || !gamma_q || !gamma_k || !q_out || !k_cache || !v_cache)
-        return WF_ERR_INVALID_ARG;
+    if (!q || !k || !v || !gamma_q || !gamma_k || !k_cache || !v_cache) return WF_ERR_INVALID_ARG;
+    if (q8 == nullptr && !q_out) return WF_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_out) ||
         !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(gamma_q) || !aligned16(gamma_k))
+        return WF_ERR_INVALID_ARG;
+    if (q8 != nullptr && (!aligned16(q8) || !q_scale || !aligned4(q_scale)))
         return WF_ERR_INVALID_ARG;
     if (pos_thw == nullptr && p->rope.F == 0) return WF_ERR_INVALID_ARG;
     if (pos_thw != nullptr && (reinterpret_cast<uintptr_t>(pos_thw) & 3u)) return WF_ERR_INVALID_ARG;
@@ -341,6 +344,8 @@ int wf_qk_norm_rope_append(wf_plan_t p, long round, const void *q, const void *k
     a.gamma_q = gamma_q;
     a.gamma_k = gamma_k;
     a.q_out = static_cast<uint16_t *>(q_out);
+    a.q8 = q8;
+    a.q_scale = q_scale;
     a.k_cache = static_cast<uint16_t *>(k_cache);
     a.v_cache = static_cast<uint16_t *>(v_cache);
     a.round = round;
@@ -352,6 +357,26 @@ int wf_qk_norm_rope_append(wf_plan_t p, long round, const void *q, const void *k
     a.rope = p->rope;
     cudaError_t e = wf::launch_append(a, p->D, static_cast<cudaStream_t>(stream), p->words);
     return e == cudaSuccess ? WF_OK : WF_ERR_CUDA;
+}
+
+int wf_qk_norm_rope_append(wf_plan_t p, long round, const void *q, const void *k, const void *v,
+                           const int32_t *pos_thw, const float *gamma_q, const float *gamma_k,
+                           void *q_out, void *k_cache, void *v_cache, void *stream)
+{
+    wf::NvtxRange nvtx_range("wf_qk_norm_rope_append");
+    return append_common(p, round, q, k, v, pos_thw, gamma_q, gamma_k, q_out, nullptr, nullptr,
+                         k_cache, v_cache, stream);
+}
+
+int wf_qk_norm_rope_append_fp8q(wf_plan_t p, long round, const void *q, const void *k,
+                                const void *v, const int32_t *pos_thw, const float *gamma_q,
+                                const float *gamma_k, void *q_out, void *q8, float *q_scale,
+                                void *k_cache, void *v_cache, void *stream)
+{
+    wf::NvtxRange nvtx_range("wf_qk_norm_rope_append_fp8q");
+    if (q8 == nullptr) return WF_ERR_INVALID_ARG;
+    return append_common(p, round, q, k, v, pos_thw, gamma_q, gamma_k, q_out,
+                         static_cast<uint8_t *>(q8), q_scale, k_cache, v_cache, stream);
 }
 
 int wf_chunk_causal_attn(wf_plan_t p, long round, const void *q_out, const void *k_cache,

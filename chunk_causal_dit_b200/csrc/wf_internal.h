@@ -61,7 +61,9 @@ struct AppendParams {
     const uint16_t *q, *k, *v;
     const int32_t *pos;       // [T,3] or nullptr (derive)
     const float *gamma_q, *gamma_k;
-    uint16_t *q_out, *k_cache, *v_cache;
+    uint16_t *q_out, *k_cache, *v_cache;   // q_out may be nullptr when q8 is set
+    uint8_t *q8;              // fused FP8 Q: E4M3 codes [T,H,D] of bf16(q'), or nullptr
+    float *q_scale;           // fused FP8 Q: [H][T] per-row scales
     long round;
     int L, W, R, H;
     int heads_per_block;      // heads covered by one block (blockIdx.y picks the group)

@@ -9,8 +9,9 @@ the binding in ``chunk_causal_dit_b200.wf``.
 Per round i (staging slot s = i % 2):
   copy-in stream : q, k, v host -> device slot s   (after round i-2 released s)
   compute stream : wf_qk_norm_rope_append, wf_chunk_causal_attn (after copy-in);
-                   with the FP8 Q.K^T variant: append, wf_quantize_q_fp8,
-                   wf_quantize_k_fp8 of the wave's chunks, wf_chunk_causal_attn_fp8qk
+                   with the FP8 Q.K^T variant: the append with fused Q quantization
+                   (wf_qk_norm_rope_append_fp8q), wf_quantize_k_fp8 of the wave's chunks,
+                   wf_chunk_causal_attn_fp8qk
   copy-out stream: O device slot s -> host         (after the attention)
 """
 from __future__ import annotations
@@ -91,16 +92,20 @@ class HostRoundPipeline:
             c = self.s_comp
             c.wait_event(self.in_ready[slot])
             c.wait_event(self.o_free[slot])
-            wf.wf_qk_norm_rope_append(self.plan, r, self.q[slot], self.k[slot], self.v[slot],
-                                      self.pos, self.gq, self.gk, self.q_out, self.kc, self.vc,
-                                      c)
-            self.in_free[slot].record(c)
             if self.fp8 is None:
+                wf.wf_qk_norm_rope_append(self.plan, r, self.q[slot], self.k[slot], self.v[slot],
+                                          self.pos, self.gq, self.gk, self.q_out, self.kc,
+                                          self.vc, c)
+                self.in_free[slot].record(c)
                 wf.wf_chunk_causal_attn(self.plan, r, self.q_out, self.kc, self.vc,
                                         self.o[slot], None, c)
             else:
+                # the append writes q's E4M3 codes itself (no bf16 q_out round trip)
                 k8, ks = self.fp8
-                wf.wf_quantize_q_fp8(self.plan, self.q_out, self.q8, self.q_scale, c)
+                wf.wf_qk_norm_rope_append_fp8q(self.plan, r, self.q[slot], self.k[slot],
+                                               self.v[slot], self.pos, self.gq, self.gk, None,
+                                               self.q8, self.q_scale, self.kc, self.vc, c)
+                self.in_free[slot].record(c)
                 wf.wf_quantize_k_fp8(self.plan, r, self.plan.W, self.kc, k8, ks, c)
                 wf.wf_chunk_causal_attn_fp8qk(self.plan, r, self.q8, self.q_scale, k8, ks,
                                               self.vc, self.o[slot], None, c)

@@ -56,6 +56,8 @@ SIGNATURES = {
     "wf_status_string": (ctypes.c_char_p, [_I]),
     "wf_chunk_causal_attn_noalloc": (_I, [_I, _I, _I, _I, _I, _L, _P, _P, _P, _P, _P, _P]),
     "wf_quantize_q_fp8": (_I, [_P, _P, _P, _P, _P]),
+    "wf_qk_norm_rope_append_fp8q": (_I, [_P, _L, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                         _P]),
     "wf_quantize_k_fp8": (_I, [_P, _L, _I, _P, _P, _P, _P]),
     "wf_chunk_causal_attn_fp8qk": (_I, [_P, _L, _P, _P, _P, _P, _P, _P, _P, _P]),
     "wf_linear": (_I, [_P, _I, _I, _I, _P, _P, _P, _I, _P, _P, _I, _P, _P]),
@@ -210,6 +212,16 @@ def wf_quantize_q_fp8(plan: Plan, q_out, q8, q_scale, stream=None) -> None:
     """q_out [T,H,D] bf16 -> q8 [T,H,D] uint8 E4M3 codes, q_scale [H,T] float32."""
     _check(load().wf_quantize_q_fp8(plan.handle, _ptr(q_out), _ptr(q8), _ptr(q_scale),
                                     _stream(stream)), "wf_quantize_q_fp8")
+
+
+def wf_qk_norm_rope_append_fp8q(plan: Plan, round_: int, q, k, v, pos_thw, gamma_q, gamma_k,
+                                q_out, q8, q_scale, k_cache, v_cache, stream=None) -> None:
+    """wf_qk_norm_rope_append that also writes the E4M3 codes q8 [T,H,D] uint8 and
+    row scales q_scale [H,T] float32 of its bf16 q'; q_out may be None."""
+    _check(load().wf_qk_norm_rope_append_fp8q(
+        plan.handle, round_, _ptr(q), _ptr(k), _ptr(v), _ptr(pos_thw), _ptr(gamma_q),
+        _ptr(gamma_k), _ptr(q_out), _ptr(q8), _ptr(q_scale), _ptr(k_cache), _ptr(v_cache),
+        _stream(stream)), "wf_qk_norm_rope_append_fp8q")
 
 
 def wf_quantize_k_fp8(plan: Plan, first_chunk: int, n_chunks: int, k_cache, k8_cache, k_scale,

@@ -191,6 +191,21 @@ WF_API int wf_chunk_causal_attn(wf_plan_t plan, long round,
 WF_API int wf_quantize_q_fp8(wf_plan_t plan, const void *q_out, void *q8, float *q_scale,
                              void *stream);
 
+/* wf_qk_norm_rope_append with the row quantization of wf_quantize_q_fp8 fused
+ * into the same pass: q8 [T,H,D] E4M3 codes and q_scale [H,T] are exactly what
+ * wf_quantize_q_fp8 writes for the bf16 q_out this call computes (same rule,
+ * same bits), and K'/V go to the ring as in wf_qk_norm_rope_append.  q_out may
+ * be NULL (the FP8 attention reads only q8), which saves its write.  Device
+ * pointers: q, k, v, q_out, q8 and the caches 16-byte aligned, q_scale 4-byte
+ * aligned.  One kernel launch on `stream`; per element it reads q, k, v and
+ * writes K', V and one code byte (plus q_out when given). */
+WF_API int wf_qk_norm_rope_append_fp8q(wf_plan_t plan, long round,
+                                       const void *q, const void *k, const void *v,
+                                       const int32_t *pos_thw,
+                                       const float *gamma_q, const float *gamma_k,
+                                       void *q_out, void *q8, float *q_scale,
+                                       void *k_cache, void *v_cache, void *stream);
+
 /* Quantize the K of absolute chunks first_chunk .. first_chunk+n_chunks-1, read
  * from k_cache [R,L,H,D] bf16 at slots (chunk mod R), into k8_cache [R,L,H,D]
  * (E4M3 codes, same slots) and k_scale [R, ceil(L/128), H] (fp32), one scale

@@ -196,3 +196,38 @@ def test_full_size_sampled_fp8qk(wf):
     assert np.max(np.abs(lse.cpu().numpy()[heads, rows] - lse_ref)) <= 1e-3
     assert np.isfinite(o_all).all()
     plan.destroy()
+
+
+@pytest.mark.parametrize("L,W,Hh,H,D,r,with_q_out", [(300, 4, 2, 3, 128, 5, True),
+                                                     (200, 3, 1, 2, 64, 2, True),
+                                                     (4680 // 4, 5, 2, 12, 128, 2, False)])
+def test_fused_append_quantization_bit_exact(wf, L, W, Hh, H, D, r, with_q_out):
+    """wf_qk_norm_rope_append_fp8q: the ring writes equal the plain append's bit for
+    bit, q_out (when given) too, and q8 / q_scale equal the oracle's row rule applied
+    to that bf16 q_out (and so the stand-alone wf_quantize_q_fp8 on it)."""
+    T, R = W * L, W + Hh
+    F, gh, gw = 1, 1, L                      # a row of patches per chunk: positions derived
+    x = [rand_bf16((T, H, D), 30 + i) for i in range(3)]
+    x[0][3] = 0                              # an all-zero q row: its q' is zero, scale 1
+    gq, gk = (t.cuda() for t in wi.gains(H, D, 4))
+    plan = wf.Plan(L, W, Hh, H, D).set_rope(F, gh, gw)
+    kc0 = torch.full((R, L, H, D), 1.5, dtype=torch.bfloat16, device="cuda")
+    vc0 = torch.full_like(kc0, -2.0)
+    kc1, vc1 = kc0.clone(), vc0.clone()
+    q_ref = torch.empty_like(x[0])
+    wf.wf_qk_norm_rope_append(plan, r, x[0], x[1], x[2], None, gq, gk, q_ref, kc0, vc0)
+    q_out = torch.full_like(x[0], float("nan")) if with_q_out else None
+    q8 = torch.full((T, H, D), 0xAA, dtype=torch.uint8, device="cuda")
+    qs = torch.full((H, T), -1.0, dtype=torch.float32, device="cuda")
+    wf.wf_qk_norm_rope_append_fp8q(plan, r, x[0], x[1], x[2], None, gq, gk, q_out, q8, qs, kc1, vc1)
+    torch.cuda.synchronize()
+    assert wf.wf_sync_status(plan) == wf.WF_OK
+    assert torch.equal(kc1.view(torch.int16), kc0.view(torch.int16))
+    assert torch.equal(vc1.view(torch.int16), vc0.view(torch.int16))
+    if with_q_out:
+        assert torch.equal(q_out.view(torch.int16), q_ref.view(torch.int16))
+    rq8, rqs = oracle.quantize_rows_fp8(_bits(q_ref))
+    assert np.array_equal(q8.cpu().numpy(), rq8)
+    assert np.array_equal(qs.cpu().numpy(), rqs)
+    assert float(qs[0, 3]) == 1.0            # the zero row
+    plan.destroy()
