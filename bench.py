@@ -656,6 +656,102 @@ def measure_round_loop(w, rounds, warmup, dev, peaks, seed=0, dist=None):
                 "clocks": clocks.summary(t0, t1)}}
 
 
+VAE_STAGE = dict(T=12, H=120, W=208, C=384)
+
+
+def measure_vae_stage(steps, warmup, dev, peaks, seed=0):
+    """The streaming VAE-decode stage: one residual block (RMSNorm + SiLU, causal
+    3x3x3 conv, RMSNorm + SiLU, causal conv + residual) per chunk of 12 frames at
+    120 x 208 with 384 channels, chunk after chunk, each convolution reading the
+    previous chunk's last two input frames as its history (views into the
+    previous chunk's buffers: double-buffered, no copies).  CUDA events around
+    every kernel; the convolutions' roofline is the bf16 tensor peak (burst)."""
+    import torch
+    from chunk_causal_dit_b200 import wf
+    T, H, W, C = VAE_STAGE["T"], VAE_STAGE["H"], VAE_STAGE["W"], VAE_STAGE["C"]
+    stream = torch.cuda.current_stream(dev)
+    plan = wf.Plan(64, 1, 0, 1, 128)
+    xs = [wi.bf16_normal((T, H, W, C), seed + i, wi.STREAM_X).to(dev) for i in range(2)]
+    w1 = wi.bf16_weight(C, 27 * C, seed, 1).reshape(C, 3, 3, 3, C).contiguous().to(dev)
+    w2 = wi.bf16_weight(C, 27 * C, seed, 2).reshape(C, 3, 3, 3, C).contiguous().to(dev)
+    b1 = wi.f32_vector((C,), 0.02, seed, wi.STREAM_BIAS, 1).to(dev)
+    b2 = wi.f32_vector((C,), 0.02, seed, wi.STREAM_BIAS, 2).to(dev)
+    g1 = (1 + 0.1 * wi.f32_vector((C,), 1.0, seed, wi.STREAM_GAMMA, 1)).to(dev)
+    g2 = (1 + 0.1 * wi.f32_vector((C,), 1.0, seed, wi.STREAM_GAMMA, 2)).to(dev)
+    h1 = [torch.empty((T, H, W, C), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    h2 = [torch.empty_like(h1[0]) for _ in range(2)]
+    c1 = torch.empty_like(h1[0])
+    out = torch.empty_like(h1[0])
+
+    def chunk(i, ev=None):
+        a, prev = i % 2, (i + 1) % 2
+        hist1 = h1[prev][T - 2:] if i > 0 else None
+        hist2 = h2[prev][T - 2:] if i > 0 else None
+        x = xs[i % 2]
+        if ev is not None:
+            ev[0].record(stream)
+        wf.wf_rms_norm_silu(plan, x, g1, h1[a], stream)
+        if ev is not None:
+            ev[1].record(stream)
+        wf.wf_causal_conv3d(plan, h1[a], hist1, w1, b1, None, c1, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        wf.wf_rms_norm_silu(plan, c1, g2, h2[a], stream)
+        if ev is not None:
+            ev[3].record(stream)
+        wf.wf_causal_conv3d(plan, h2[a], hist2, w2, b2, x, out, stream)
+        if ev is not None:
+            ev[4].record(stream)
+
+    for i in range(warmup):
+        chunk(i)
+    torch.cuda.synchronize(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    clocks = ClockSampler(dev.index)
+    time.sleep(0.02)
+    torch.cuda.synchronize(dev)
+    t0 = time.time()
+    for i in range(steps):
+        chunk(warmup + i, ev[i])
+    torch.cuda.synchronize(dev)
+    t1 = time.time()
+    clocks.stop()
+    status = wf.wf_sync_status(plan, stream)
+    plan.destroy()
+    if status != wf.WF_OK:
+        raise SystemExit("device status %d (%s) in the VAE leg" % (status, wf.status_string(status)))
+    conv_flop = 2.0 * T * H * W * C * C * 27      # every tap of the 3x3x3 kernel
+    norm_ms = statistics.mean(e[0].elapsed_time(e[1]) + e[2].elapsed_time(e[3]) for e in ev) / 2
+    conv_ms = statistics.mean(e[1].elapsed_time(e[2]) + e[3].elapsed_time(e[4]) for e in ev) / 2
+    blk_ms = statistics.mean(e[0].elapsed_time(e[4]) for e in ev)
+    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    conv_tf = conv_flop / (conv_ms * 1e-3) / 1e12
+    norm_bytes = 4 * T * H * W * C
+    return {
+        "what": "streaming VAE-decode stage: residual block (RMSNorm+SiLU, causal 3x3x3 conv, "
+                "RMSNorm+SiLU, causal conv + residual) per chunk, history from the previous chunk",
+        "frames_per_chunk": T, "height": H, "width": W, "channels": C,
+        "steps": steps, "warmup": warmup,
+        "block_ms_per_chunk": round(blk_ms, 4),
+        "chunks_per_s": round(1e3 / blk_ms, 2),
+        "frames_per_s": round(T * 1e3 / blk_ms, 1),
+        "block_tflops": round(2 * conv_flop / (blk_ms * 1e-3) / 1e12, 2),
+        "conv": {"kernel": "gemm_pair_kernel<conv, BN=192> (implicit GEMM, K = 27 taps x 384)",
+                 "bound": "tensor", "ms_per_launch": round(conv_ms, 5),
+                 "achieved": round(conv_tf, 2), "peak": peak, "unit": "TFLOP/s",
+                 "frac": round(conv_tf / peak, 4),
+                 "frac_nominal": round(conv_tf / NOMINAL_BF16_TFLOPS, 4),
+                 "flop_per_launch": conv_flop},
+        "norm": {"kernel": "rms_norm_silu_kernel", "bound": "hbm",
+                 "ms_per_launch": round(norm_ms, 5),
+                 "achieved": round(norm_bytes / (norm_ms * 1e-3) / 1e9, 1), "peak": hbm,
+                 "unit": "GB/s", "frac": round(norm_bytes / (norm_ms * 1e-3) / 1e9 / hbm, 4),
+                 "bytes_per_launch": norm_bytes},
+        "clocks": clocks.summary(t0, t1),
+    }
+
+
 def run_config_legs(args, dev, peaks):
     """The other configurations of the benchmark, each a short leg with its own
     clock record: the tiny wave (latency), the 5-step and 14B waves, the 30-layer
@@ -670,6 +766,8 @@ def run_config_legs(args, dev, peaks):
                                               peaks)["summary"]
     torch.cuda.empty_cache()
     fp8 = measure_single_layer(wi.WORKLOADS[args.workload], 30, 5, dev, peaks, fp8=True)
+    torch.cuda.empty_cache()
+    legs["vae_stage"] = measure_vae_stage(10, 3, dev, peaks)
     torch.cuda.empty_cache()
     return legs, fp8
 

@@ -26,7 +26,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libwf.so")
 LIB_CHECK = os.path.join(HERE, "libwf_check.so")
 SOURCES = ["wf_api.cu", "append_kernel.cu", "attn_kernel.cu", "attn_pair_kernel.cu",
-           "quant_fp8_kernel.cu", "noalloc.cu", "gemm_kernel.cu", "ln_kernel.cu"]
+           "quant_fp8_kernel.cu", "noalloc.cu", "gemm_kernel.cu", "ln_kernel.cu", "vae_kernel.cu"]
 HEADERS = ["sm100.cuh", "wf_internal.h", "exp2_poly.h", "wf_check.cuh", "fp8_rule.cuh"]
 
 NVCC_FLAGS = [

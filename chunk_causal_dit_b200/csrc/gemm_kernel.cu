@@ -46,13 +46,25 @@ namespace wf {
 namespace {
 
 constexpr int BM = 128;                    // rows of A per CTA (M = 256 per pair MMA)
-constexpr int BN = 256;                    // columns of C per tile (the MMA's N)
 constexpr int BK = 64;                     // K per stage: one 128-byte swizzle row of bf16
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 32 * (2 + kEpiWarps);   // producer, MMA, 8 epilogue warps
 constexpr uint32_t kABytes = BM * BK * 2;              // 16 KB
-constexpr uint32_t kBBytes = (BN / 2) * BK * 2;        // 16 KB: this CTA's 128 rows of B
-constexpr uint32_t kStageBytes = kABytes + kBBytes;
+
+// Tile width BN (columns of C per tile, the MMA's N): 256 for the linear layers;
+// the convolution takes 192 when the output channels are a multiple of it (384
+// and 192 fill whole tiles).  Each CTA holds BN / 2 rows of B per stage.
+template <int BN>
+struct Tile {
+    static_assert(BN == 256 || BN == 192, "tile width");
+    static constexpr uint32_t kBBytes = (BN / 2) * BK * 2;
+    static constexpr uint32_t kStageBytes = kABytes + kBBytes;
+};
+
+template <int Epi>
+struct IsConv {
+    static constexpr bool value = Epi == kEpiConv || Epi == kEpiConvResidual;
+};
 constexpr int kTabMax = 3072;                          // float2 entries (24 KB)
 constexpr uint32_t kStageRowBytes = 80;                // epilogue staging (see warp_store32)
 constexpr uint32_t kWarpStageBytes = 32 * kStageRowBytes;
@@ -62,9 +74,10 @@ constexpr unsigned long long kDrainLimit = 1ull << 32;
 // Shared-memory plan per epilogue: the stage ring, then (QKV only) the RoPE
 // (cos, sin) tables, the epilogue warps' staging buffers and the barrier block.
 // (Six stages measured 1-4% faster than seven; with the tables only five fit.)
-template <int Epi>
+template <int Epi, int BN>
 struct Smem {
-    static constexpr int kStages = Epi == kEpiQkvAppend ? 5 : 6;
+    static constexpr uint32_t kStageBytes = Tile<BN>::kStageBytes;
+    static constexpr int kStages = Epi == kEpiQkvAppend ? 5 : (BN == 192 ? 7 : 6);
     static constexpr uint32_t kTabOff = kStages * kStageBytes;
     static constexpr uint32_t kStgOff = kTabOff + (Epi == kEpiQkvAppend ? kTabMax * 8 : 0);
     static constexpr uint32_t kBarOff = kStgOff + kEpiWarps * kWarpStageBytes;
@@ -214,6 +227,17 @@ __device__ __forceinline__ void finish32(const GemmParams &p, const uint32_t (&r
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = gelu_tanh(v[i]);
     }
+    if constexpr (Epi == kEpiConvResidual) {
+        uint4 rw[4];
+        warp_load32(stage, row_ok ? p.resid + row * p.N + c : nullptr, rw);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float x[8];
+            unpack8(rw[j], x);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[8 * j + e] += x[e];
+        }
+    }
     if constexpr (Epi == kEpiGatedResidual) {
         uint4 rw[4];
         warp_load32(stage, row_ok ? p.resid + row * p.N + c : nullptr, rw);
@@ -235,17 +259,18 @@ __device__ __forceinline__ void finish32(const GemmParams &p, const uint32_t (&r
     warp_store32(stage, w, st ? p.c + row * p.N + c : nullptr);
 }
 
-// Linear epilogues: this thread's row, 128 columns from col0 (TMEM at taddr).
-template <int Epi>
-__device__ __forceinline__ void epi_linear(const GemmParams &p, uint32_t taddr, long row, int col0,
-                                           uint8_t *stage)
+// Linear and convolution epilogues: this thread's row (row_ok: it exists), kCols
+// columns from col0 (TMEM at taddr), in pairs of 32-column chunks.
+template <int Epi, int kCols>
+__device__ __forceinline__ void epi_linear(const GemmParams &p, uint32_t taddr, long row,
+                                           bool row_ok, int col0, uint8_t *stage)
 {
-    const bool row_ok = row < p.M;
+    static_assert(kCols % 32 == 0, "32-column chunks");
     const float *gate_row = nullptr;
     if constexpr (Epi == kEpiGatedResidual)
         gate_row = p.gate + (row_ok ? row / p.rows_per_group : 0) * static_cast<long>(p.N);
 #pragma unroll 1
-    for (int h = 0; h < 2; ++h) {
+    for (int h = 0; h < kCols / 64; ++h) {
         uint32_t r0[32], r1[32];
         tmem_ld32(taddr + 64 * h, r0);
         tmem_ld32(taddr + 64 * h + 32, r1);
@@ -254,6 +279,35 @@ __device__ __forceinline__ void epi_linear(const GemmParams &p, uint32_t taddr, 
         if (c < p.N) finish32<Epi>(p, r0, row, row_ok, c, gate_row, stage);
         if (c + 32 < p.N) finish32<Epi>(p, r1, row, row_ok, c + 32, gate_row, stage);
     }
+    if constexpr (kCols % 64 != 0) {
+        uint32_t r0[32];
+        const int h = kCols / 64;
+        tmem_ld32(taddr + 64 * h, r0);
+        tmem_wait_ld();
+        const int c = col0 + 64 * h;
+        if (c < p.N) finish32<Epi>(p, r0, row, row_ok, c, gate_row, stage);
+    }
+}
+
+// Output pixel of a convolution tile: tile t (column tile fastest, then 16-column
+// and 16-row pixel tiles, then frames), CTA rank r (rows 8r .. 8r + 7 of the
+// tile) and row m of the CTA's 128 rows (16 pixels per row).
+struct ConvTile {
+    int nb, f, y0, x0;
+};
+
+__device__ __forceinline__ ConvTile conv_tile(const GemmParams &p, int t)
+{
+    ConvTile c;
+    c.nb = t % p.n_ntiles;
+    int rest = t / p.n_ntiles;
+    const int px = rest % p.n_px;
+    rest /= p.n_px;
+    const int py = rest % p.n_py;
+    c.f = rest / p.n_py;
+    c.x0 = px * 16;
+    c.y0 = py * 16;
+    return c;
 }
 
 // QKV epilogue: this thread's wave token `row`, 128 columns from col0, i.e. 128 / D
@@ -375,13 +429,15 @@ __device__ __forceinline__ void epi_qkv(const GemmParams &p, uint32_t taddr, lon
     }
 }
 
-template <int Epi, int D>
+template <int Epi, int D, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                 const __grid_constant__ GemmParams p)
+                 const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ GemmParams p)
 {
-    using B = Smem<Epi>;
+    using B = Smem<Epi, BN>;
     constexpr int kStages = B::kStages;
+    constexpr uint32_t kStageBytes = Tile<BN>::kStageBytes;
+    constexpr bool kConv = IsConv<Epi>::value;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -398,7 +454,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     const int cid = static_cast<int>(cluster_id_x());
     const int ncl = static_cast<int>(nclusters_x());
     auto lead = [&](int i) -> uint32_t { return map_to_rank(bar(i), 0); };
-    const int nk = (p.K + BK - 1) / BK;
+    // K slices: one per 64 columns of K, or per (tap, 64 input channels) of a conv
+    const int nk = kConv ? 27 * p.n_cblk : (p.K + BK - 1) / BK;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -461,13 +518,23 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
             // ---------------- TMA producer (both CTAs) ----------------
             tma_prefetch_desc(&tmap_a);
             tma_prefetch_desc(&tmap_b);
+            if (kConv && p.use_hist) tma_prefetch_desc(&tmap_h);
             uint32_t it = 0;
             const bool withheld = p.withhold != 0;   // test hook: stage 0's first fill never comes
             bool ok = true;
             for (int t = cid; ok && t < p.n_tiles; t += ncl) {
-                const int mb = t / p.n_ntiles, nb = t - mb * p.n_ntiles;
-                const int arow = mb * 2 * BM + static_cast<int>(rank) * BM;
-                const int brow = nb * BN + static_cast<int>(rank) * (BN / 2);
+                int arow = 0, brow = 0, fr = 0, ya = 0, xa = 0;
+                if constexpr (kConv) {
+                    const ConvTile ct = conv_tile(p, t);
+                    brow = ct.nb * BN + static_cast<int>(rank) * (BN / 2);
+                    fr = ct.f;
+                    ya = ct.y0 + 8 * static_cast<int>(rank);
+                    xa = ct.x0;
+                } else {
+                    const int mb = t / p.n_ntiles, nb = t - mb * p.n_ntiles;
+                    arow = mb * 2 * BM + static_cast<int>(rank) * BM;
+                    brow = nb * BN + static_cast<int>(rank) * (BN / 2);
+                }
                 for (int kb = 0; kb < nk; ++kb, ++it) {
                     const uint32_t st = it % kStages;
                     if (!(ok = wait_bar(bar(B::empty + st), ((it / kStages) & 1u) ^ 1u, ctl,
@@ -476,8 +543,24 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                     if (withheld && it == 0) continue;
                     if (leader) mbar_arrive_expect_tx(bar(B::full + st), 2 * kStageBytes);
                     const uint32_t dst = sbase + st * kStageBytes;
-                    tma_load_2d_pair(dst, &tmap_a, lead(B::full + st), kb * BK, arow);
-                    tma_load_2d_pair(dst + kABytes, &tmap_b, lead(B::full + st), kb * BK, brow);
+                    if constexpr (kConv) {
+                        // tap (dt, dy, dx), channels [64 cb, 64 cb + 64): A is the 16 x 8
+                        // pixel box shifted by the tap (rows and columns outside the frame
+                        // read zeros); taps before the chunk read the history's frame
+                        // tf + 2, or zeros at the start of the video
+                        const int tap = kb / p.n_cblk, cb = kb - tap * p.n_cblk;
+                        const int dt = tap / 9, dy = (tap / 3) % 3, dx = tap % 3;
+                        const int tf = fr + dt - 2;
+                        const bool hist = tf < 0 && p.use_hist;
+                        tma_load_4d_pair(dst, hist ? &tmap_h : &tmap_a, lead(B::full + st),
+                                         cb * BK, xa + dx - 1, ya + dy - 1, hist ? tf + 2 : tf);
+                        tma_load_3d_pair(dst + kABytes, &tmap_b, lead(B::full + st), cb * BK, tap,
+                                         brow);
+                    } else {
+                        tma_load_2d_pair(dst, &tmap_a, lead(B::full + st), kb * BK, arow);
+                        tma_load_2d_pair(dst + kABytes, &tmap_b, lead(B::full + st), kb * BK,
+                                         brow);
+                    }
                 }
             }
             if (!ok && leader) {
@@ -539,15 +622,30 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
             ok = __all_sync(0xFFFFFFFFu, ok);
             if (!ok) break;
             tc_fence_after();
-            const int mb = t / p.n_ntiles, nb = t - mb * p.n_ntiles;
-            const long row = static_cast<long>(mb) * 2 * BM + rank * BM + lq * 32 + lane;
+            long row;
+            bool row_ok;
+            int nb;
+            if constexpr (kConv) {
+                const ConvTile ct = conv_tile(p, t);
+                const int m = lq * 32 + lane;
+                const int y = ct.y0 + 8 * static_cast<int>(rank) + (m >> 4);
+                const int x = ct.x0 + (m & 15);
+                nb = ct.nb;
+                row_ok = y < p.ch && x < p.cw;
+                row = (static_cast<long>(ct.f) * p.ch + y) * p.cw + x;
+            } else {
+                const int mb = t / p.n_ntiles;
+                nb = t - mb * p.n_ntiles;
+                row = static_cast<long>(mb) * 2 * BM + rank * BM + lq * 32 + lane;
+                row_ok = row < p.M;
+            }
             const int col0 = nb * BN + half * (BN / 2);
             const uint32_t taddr =
                 tmem + (static_cast<uint32_t>(lq * 32) << 16) + b * BN + half * (BN / 2);
             if constexpr (Epi == kEpiQkvAppend)
                 epi_qkv<D>(p, taddr, row, col0, tab, stage);
             else
-                epi_linear<Epi>(p, taddr, row, col0, stage);
+                epi_linear<Epi, BN / 2>(p, taddr, row, row_ok, col0, stage);
             // the accumulator may be overwritten once this warp's TMEM loads are done
             // (tcgen05.wait::ld above): a relaxed arrive, so that the epilogue's global
             // stores need not drain first, as a release at cluster scope would demand
@@ -568,14 +666,14 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     }
 }
 
-template <int Epi, int D>
-cudaError_t launch_gemm_t(const CUtensorMap &ma, const CUtensorMap &mb, const GemmParams &p,
-                          cudaStream_t stream)
+template <int Epi, int D, int BN = 256>
+cudaError_t launch_gemm_t(const CUtensorMap &ma, const CUtensorMap &mb, const CUtensorMap &mh,
+                          const GemmParams &p, cudaStream_t stream)
 {
     constexpr int kMaxDevices = 64;
     static std::atomic<int> resident_pairs[kMaxDevices];
-    auto kern = gemm_pair_kernel<Epi, D>;
-    constexpr uint32_t smem = Smem<Epi>::kBytes;
+    auto kern = gemm_pair_kernel<Epi, D, BN>;
+    constexpr uint32_t smem = Smem<Epi, BN>::kBytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -604,7 +702,7 @@ cudaError_t launch_gemm_t(const CUtensorMap &ma, const CUtensorMap &mb, const Ge
     }
     const int n_clusters = p.n_tiles < resident ? p.n_tiles : resident;
     cfg.gridDim = dim3(2 * n_clusters, 1, 1);
-    e = cudaLaunchKernelEx(&cfg, kern, ma, mb, p);
+    e = cudaLaunchKernelEx(&cfg, kern, ma, mb, mh, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -618,14 +716,29 @@ cudaError_t launch_gemm(const CUtensorMap &ma, const CUtensorMap &mb, const Gemm
 {
     if (p.n_tiles == 0) return cudaSuccess;
     switch (epi) {
-    case kEpiStore: return launch_gemm_t<kEpiStore, 128>(ma, mb, p, stream);
-    case kEpiGeluTanh: return launch_gemm_t<kEpiGeluTanh, 128>(ma, mb, p, stream);
-    case kEpiGatedResidual: return launch_gemm_t<kEpiGatedResidual, 128>(ma, mb, p, stream);
+    case kEpiStore: return launch_gemm_t<kEpiStore, 128>(ma, mb, ma, p, stream);
+    case kEpiGeluTanh: return launch_gemm_t<kEpiGeluTanh, 128>(ma, mb, ma, p, stream);
+    case kEpiGatedResidual: return launch_gemm_t<kEpiGatedResidual, 128>(ma, mb, ma, p, stream);
     case kEpiQkvAppend:
-        return p.D == 128 ? launch_gemm_t<kEpiQkvAppend, 128>(ma, mb, p, stream)
-                          : launch_gemm_t<kEpiQkvAppend, 64>(ma, mb, p, stream);
+        return p.D == 128 ? launch_gemm_t<kEpiQkvAppend, 128>(ma, mb, ma, p, stream)
+                          : launch_gemm_t<kEpiQkvAppend, 64>(ma, mb, ma, p, stream);
     default: return cudaErrorInvalidValue;
     }
+}
+
+// Causal 3x3x3 convolution as an implicit GEMM: mx over the chunk [ct][ch][cw][cin]
+// and mh over its two history frames (box 64 channels x 16 columns x 8 rows x 1
+// frame), mw over the weights [N][27][cin] (box 64 x 1 x BN / 2), 128-byte swizzle.
+// bn: the tile width the maps were encoded for (192 or 256).
+cudaError_t launch_conv(const CUtensorMap &mx, const CUtensorMap &mh, const CUtensorMap &mw,
+                        const GemmParams &p, bool residual, int bn, cudaStream_t stream)
+{
+    if (p.n_tiles == 0) return cudaSuccess;
+    if (bn == 192)
+        return residual ? launch_gemm_t<kEpiConvResidual, 128, 192>(mx, mw, mh, p, stream)
+                        : launch_gemm_t<kEpiConv, 128, 192>(mx, mw, mh, p, stream);
+    return residual ? launch_gemm_t<kEpiConvResidual, 128, 256>(mx, mw, mh, p, stream)
+                    : launch_gemm_t<kEpiConv, 128, 256>(mx, mw, mh, p, stream);
 }
 
 int gemm_tab_max() { return kTabMax; }

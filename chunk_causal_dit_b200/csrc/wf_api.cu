@@ -32,6 +32,11 @@ cudaError_t launch_layer_norm_modulate(const uint16_t *x, const float *shift, co
                                        uint16_t *y, long M, int C, int rows_per_group, float eps,
                                        cudaStream_t stream);
 int ln_max_channels();
+cudaError_t launch_conv(const CUtensorMap &mx, const CUtensorMap &mh, const CUtensorMap &mw,
+                        const GemmParams &p, bool residual, int bn, cudaStream_t stream);
+cudaError_t launch_rms_norm_silu(const uint16_t *x, const float *gamma, uint16_t *y, long M, int C,
+                                 float eps, cudaStream_t stream);
+int rms_norm_silu_max_channels();
 }  // namespace wf
 
 namespace wf {
@@ -150,6 +155,40 @@ bool encode_map_2d(CUtensorMap *map, const void *base, long rows, long cols)
                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+// 4-D map over a channels-last video [T][H][W][C] bf16: box = 64 channels x 16
+// columns x 8 rows x 1 frame (128 pixels, one 128-byte swizzle row each); reads
+// outside the frame or before the first frame return zeros.
+bool encode_map_video(CUtensorMap *map, const void *base, int T, int H, int W, int C)
+{
+    auto enc = wf::tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(W),
+                                static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
+    const cuuint64_t pix = static_cast<cuuint64_t>(C) * 2;
+    const cuuint64_t strides[3] = {pix, pix * W, pix * W * H};
+    const cuuint32_t box[4] = {64, 16, 8, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D map over conv weights [Cout][27][Cin] bf16: box = 64 channels x 1 tap x rows
+// output channels.
+bool encode_map_convw(CUtensorMap *map, const void *base, int Cout, int Cin, int rows)
+{
+    auto enc = wf::tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(Cin), 27, static_cast<cuuint64_t>(Cout)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(Cin) * 2,
+                                   static_cast<cuuint64_t>(Cin) * 2 * 27};
+    const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(rows)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Tile counts of a GEMM (256 x 256 tiles); false if they do not fit an int.
@@ -599,6 +638,70 @@ int wf_layer_norm_modulate(wf_plan_t p, int M, int C, const void *x, const float
     cudaError_t e = wf::launch_layer_norm_modulate(
         static_cast<const uint16_t *>(x), shift, scale, static_cast<uint16_t *>(y), M, C,
         rows_per_group, 1e-6f, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? WF_OK : WF_ERR_CUDA;
+}
+
+int wf_causal_conv3d(wf_plan_t p, int T, int H, int W, int Cin, int Cout, const void *x,
+                     const void *x_hist, const void *w, const float *bias, const void *resid,
+                     void *y, void *stream)
+{
+    wf::NvtxRange nvtx_range("wf_causal_conv3d");
+    if (p == nullptr || T < 1 || H < 1 || W < 1 || Cin < 8 || Cin % 8 || Cout < 32 || Cout % 32)
+        return WF_ERR_INVALID_ARG;
+    const long long M = static_cast<long long>(T) * H * W;
+    if (M >= INT_MAX || static_cast<long long>(Cin) * 27 >= INT_MAX) return WF_ERR_INVALID_ARG;
+    if (!x || !w || !y || !aligned16(x) || !aligned16(x_hist) || !aligned16(w) || !aligned16(y) ||
+        !aligned16(bias) || !aligned16(resid))
+        return WF_ERR_INVALID_ARG;
+    if (int s = check_device(p)) return s;
+
+    const int bn = Cout % 192 == 0 ? 192 : 256;
+    wf::GemmParams g{};
+    g.M = static_cast<int>(M);
+    g.N = Cout;
+    g.K = 27 * Cin;
+    g.ct = T;
+    g.ch = H;
+    g.cw = W;
+    g.cin = Cin;
+    g.n_cblk = (Cin + 63) / 64;
+    g.n_py = (H + 15) / 16;
+    g.n_px = (W + 15) / 16;
+    g.n_ntiles = (Cout + bn - 1) / bn;
+    const long long tiles = static_cast<long long>(T) * g.n_py * g.n_px * g.n_ntiles;
+    if (tiles >= INT_MAX) return WF_ERR_INVALID_ARG;
+    g.n_tiles = static_cast<int>(tiles);
+    g.use_hist = x_hist != nullptr ? 1 : 0;
+    g.bias = bias;
+    g.c = static_cast<uint16_t *>(y);
+    g.resid = static_cast<const uint16_t *>(resid);
+    g.rows_per_group = 1;
+    g.wait_limit = p->wait_limit;
+    g.withhold = p->withhold_q;
+    g.words = p->words;
+    CUtensorMap mx, mh, mw;
+    if (!encode_map_video(&mx, x, T, H, W, Cin) ||
+        !encode_map_video(&mh, x_hist != nullptr ? x_hist : x, x_hist != nullptr ? 2 : T, H, W,
+                          Cin) ||
+        !encode_map_convw(&mw, w, Cout, Cin, bn / 2))
+        return WF_ERR_CUDA;
+    cudaError_t e = wf::launch_conv(mx, mh, mw, g, resid != nullptr, bn,
+                                    static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? WF_OK : WF_ERR_CUDA;
+}
+
+int wf_rms_norm_silu(wf_plan_t p, int M, int C, const void *x, const float *gamma, void *y,
+                     void *stream)
+{
+    wf::NvtxRange nvtx_range("wf_rms_norm_silu");
+    if (p == nullptr || M < 0 || C < 8 || C % 8) return WF_ERR_INVALID_ARG;
+    if (C > wf::rms_norm_silu_max_channels()) return WF_ERR_UNSUPPORTED;
+    if (!x || !gamma || !y || !aligned16(x) || !aligned16(gamma) || !aligned16(y))
+        return WF_ERR_INVALID_ARG;
+    if (int s = check_device(p)) return s;
+    cudaError_t e = wf::launch_rms_norm_silu(static_cast<const uint16_t *>(x), gamma,
+                                             static_cast<uint16_t *>(y), M, C, 1e-6f,
+                                             static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? WF_OK : WF_ERR_CUDA;
 }
 

@@ -94,6 +94,8 @@ enum GemmEpilogue : int {
     kEpiGeluTanh = 1,         // C = gelu_tanh(A B^T + bias)
     kEpiGatedResidual = 2,    // C = resid + gate[row / rows_per_group] * (A B^T + bias)
     kEpiQkvAppend = 3,        // QKV projection: RMSNorm + RoPE on q/k, q -> q_out, k/v -> ring
+    kEpiConv = 4,             // causal 3x3x3 convolution (implicit GEMM): C = conv + bias
+    kEpiConvResidual = 5,     // the same plus a residual: C = resid + conv + bias
 };
 
 struct GemmParams {
@@ -115,6 +117,12 @@ struct GemmParams {
     unsigned long long wait_limit;
     int withhold;             // test hook: no CTA issues (or arms) its first stage's copies
     DeviceWords *words;
+    // causal 3x3x3 convolution (kEpiConv*): output [ct][ch][cw][N] with M = ct*ch*cw
+    // pixels; a K slice is one tap (dt, dy, dx) x 64 input channels
+    int ct, ch, cw, cin;
+    int n_cblk;               // 64-channel blocks of the input: ceil(cin / 64)
+    int n_py, n_px;           // 16 x 16 pixel tiles per frame (rows, columns)
+    int use_hist;             // taps before the chunk read the history map (else zeros)
 };
 
 // NVTX range around a host call of the C ABI (header-only NVTX v3: without a

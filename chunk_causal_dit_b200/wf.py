@@ -63,6 +63,8 @@ SIGNATURES = {
     "wf_linear": (_I, [_P, _I, _I, _I, _P, _P, _P, _I, _P, _P, _I, _P, _P]),
     "wf_qkv_proj_norm_rope_append": (_I, [_P, _L, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "wf_layer_norm_modulate": (_I, [_P, _I, _I, _P, _P, _P, _I, _P, _P]),
+    "wf_causal_conv3d": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
+    "wf_rms_norm_silu": (_I, [_P, _I, _I, _P, _P, _P, _P]),
 }
 
 _lib = None
@@ -295,3 +297,22 @@ def wf_chunk_causal_attn_noalloc(chunk_tokens, n_wave_chunks, n_hist_chunks, hea
                                                heads, head_dim, round_, _ptr(q_out),
                                                _ptr(k_cache), _ptr(v_cache), _ptr(o), _ptr(lse),
                                                _stream(stream)), "wf_chunk_causal_attn_noalloc")
+
+
+def wf_causal_conv3d(plan: Plan, x, x_hist, w, bias, resid, y, stream=None) -> None:
+    """Causal 3x3x3 convolution of one chunk: x [T,H,W,Cin] bf16, x_hist [2,H,W,Cin]
+    or None (start of the video), w [Cout,3,3,3,Cin] bf16, bias [Cout] f32 or None,
+    resid [T,H,W,Cout] or None, y [T,H,W,Cout] bf16."""
+    T, H, W, Cin = x.shape
+    Cout = w.shape[0]
+    _check(load().wf_causal_conv3d(plan.handle, T, H, W, Cin, Cout, _ptr(x), _ptr(x_hist),
+                                   _ptr(w), _ptr(bias), _ptr(resid), _ptr(y), _stream(stream)),
+           "wf_causal_conv3d")
+
+
+def wf_rms_norm_silu(plan: Plan, x, gamma, y, stream=None) -> None:
+    """Per-pixel RMSNorm over the last axis with gain gamma, then SiLU (bf16 in/out)."""
+    C = x.shape[-1]
+    M = x.numel() // C
+    _check(load().wf_rms_norm_silu(plan.handle, M, C, _ptr(x), _ptr(gamma), _ptr(y),
+                                   _stream(stream)), "wf_rms_norm_silu")

@@ -287,6 +287,41 @@ WF_API int wf_qkv_proj_norm_rope_append(wf_plan_t plan, long round, int hidden, 
 WF_API int wf_layer_norm_modulate(wf_plan_t plan, int M, int C, const void *x, const float *shift,
                                   const float *scale, int rows_per_group, void *y, void *stream);
 
+/* ---- The streaming VAE-decode stage -------------------------------------
+ * "Wave Forcing" (abstract) lists pipelined VAE decoding as one part of its
+ * runtime; the airadar.tv summary (usage section) takes the VAE from the Wan2.1
+ * base model, splits its decode into 2 or 3 pipeline stages (--vae-stages) and
+ * decodes 399 latent frames into 1593 video frames.  The pages print no layer
+ * of the decoder; these calls are the plain definitions of a causal 3D-conv
+ * decoder stage.  Activations are channels-last [T][H][W][C] bf16.  A video is
+ * decoded chunk by chunk: a convolution of chunk i reads, before its first
+ * frame, the last two frames of the same convolution's input in chunk i - 1,
+ * so streaming the chunks gives exactly the convolution of the whole video and
+ * the decode of one chunk can run while the next chunk is generated. */
+
+/* Causal 3x3x3 convolution of one chunk:
+ *   y[t,i,j,o] = bias[o] + sum over dt, dy, dx in 0..2 and c of
+ *                w[o][dt][dy][dx][c] * X(t+dt-2, i+dy-1, j+dx-1, c)  (+ resid[t,i,j,o])
+ * where X(tau, ...) is x for tau >= 0, x_hist[tau + 2] for tau < 0 (x_hist: the
+ * previous chunk's last two input frames [2][H][W][Cin], or NULL at the start
+ * of the video, which reads zeros), and zero outside the H x W frame.
+ * x [T][H][W][Cin], w [Cout][3][3][3][Cin], resid and y [T][H][W][Cout]: bf16
+ * device pointers, 16-byte aligned; bias [Cout] fp32 or NULL; resid may be NULL
+ * and may equal y; y must not overlap x, x_hist or w.  Cin % 8 == 0, Cout % 32
+ * == 0, T*H*W < 2^31.  bf16 tensor-core products (an implicit GEMM: K = 27 taps
+ * x Cin) with fp32 accumulation, one rounding to bf16.  One persistent kernel
+ * launch on `stream` (clusters of two CTAs). */
+WF_API int wf_causal_conv3d(wf_plan_t plan, int T, int H, int W, int Cin, int Cout,
+                            const void *x, const void *x_hist, const void *w,
+                            const float *bias, const void *resid, void *y, void *stream);
+
+/* Per pixel (row of C channels): y = x / sqrt(mean_c x^2 + 1e-6) * gamma, then
+ * y * sigmoid(y) (SiLU).  x, y [M][C] bf16, gamma [C] fp32; device pointers,
+ * 16-byte aligned; C % 8 == 0 and C <= 512 (WF_ERR_UNSUPPORTED above).  y may
+ * equal x.  fp32 arithmetic, one rounding to bf16.  One kernel launch. */
+WF_API int wf_rms_norm_silu(wf_plan_t plan, int M, int C, const void *x, const float *gamma,
+                            void *y, void *stream);
+
 /* Wait for `stream`, then read and clear the plan's device status word.
  * Returns WF_OK, WF_ERR_TIMEOUT (a bounded device wait expired), WF_ERR_BOUNDS
  * (only in the debug build libwf_check.so, compiled with -DWF_CHECK: a computed

@@ -93,14 +93,24 @@ def causal_conv3d_at(x_bits, hist_bits, w_bits, pixels, bias=None, resid_bits=No
     """:func:`causal_conv3d_f64` at selected output pixels only.
 
     pixels: int array [n, 3] of (t, i, j).  Returns (y [n, Cout] float64,
-    s [n, Cout] float64) where s = sum of |w x| over the taps (the size of the
-    terms the sum adds up, for error bars of a floating-point accumulation).
+    s [n, Cout] float64) where s = sum of |w x| over the taps plus |bias| (the
+    size of the terms the sum adds up, for error bars of a floating-point
+    accumulation).  Only the input pixels these outputs read are widened to fp64.
     """
-    xe = _extended(x_bits, hist_bits)
+    x_bits = np.asarray(x_bits, np.uint16)
+    T, H, W, _ = x_bits.shape
     w = bf16_to_f64(w_bits)
-    H, W = xe.shape[1], xe.shape[2]
     pixels = np.asarray(pixels, np.int64).reshape(-1, 3)
     Cout = w.shape[0]
+
+    def X(tau, ii, jj):
+        """Input pixel vector at frame tau (tau < 0: history frame tau + 2)."""
+        if tau < 0:
+            if hist_bits is None:
+                return None
+            return bf16_to_f64(np.asarray(hist_bits, np.uint16)[tau + KT - 1, ii, jj])
+        return bf16_to_f64(x_bits[tau, ii, jj])
+
     y = np.zeros((len(pixels), Cout))
     s = np.zeros((len(pixels), Cout))
     for n, (t, i, j) in enumerate(pixels):
@@ -108,17 +118,20 @@ def causal_conv3d_at(x_bits, hist_bits, w_bits, pixels, bias=None, resid_bits=No
             for dy in range(KS):
                 for dx in range(KS):
                     ii, jj = i + dy - 1, j + dx - 1
-                    if 0 <= ii < H and 0 <= jj < W:
-                        v = xe[t + dt, ii, jj, :]
-                        y[n] += w[:, dt, dy, dx, :] @ v
-                        s[n] += np.abs(w[:, dt, dy, dx, :]) @ np.abs(v)
+                    if not (0 <= ii < H and 0 <= jj < W):
+                        continue
+                    v = X(t + dt - (KT - 1), ii, jj)
+                    if v is None:
+                        continue
+                    y[n] += w[:, dt, dy, dx, :] @ v
+                    s[n] += np.abs(w[:, dt, dy, dx, :]) @ np.abs(v)
     if bias is not None:
         b = np.asarray(bias, np.float32).astype(np.float64)
         y += b
         s += np.abs(b)
     if resid_bits is not None:
-        r = bf16_to_f64(resid_bits)[pixels[:, 0], pixels[:, 1], pixels[:, 2]]
-        y += r
+        r = np.asarray(resid_bits, np.uint16)[pixels[:, 0], pixels[:, 1], pixels[:, 2]]
+        y += bf16_to_f64(r)
     return y, s
 
 
