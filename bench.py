@@ -752,6 +752,38 @@ def measure_vae_stage(steps, warmup, dev, peaks, seed=0):
     }
 
 
+def run_vae(args, rank, world, local):
+    """bench.py --workload vae_stage: the VAE-decode stage alone, one replica per GPU."""
+    import torch
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = make_group(world, "nccl")
+    peaks, _ = load_peaks()
+    barrier(dist, dev)
+    v = measure_vae_stage(args.steps, args.warmup, dev, peaks, seed=rank)
+    ms = allreduce_max(dist, v["block_ms_per_chunk"], dev)
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+    return {
+        "metric": "streaming VAE-decode stage: useful conv TFLOP/s (two causal 3x3x3 convs "
+                  "per chunk)",
+        "value": round(world * 2 * v["conv"]["flop_per_launch"] / (ms * 1e-3) / 1e12, 3),
+        "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded bf16 N(0,1) chunks, random-init weights)",
+        "config": {"workload": "vae_stage", "frames_per_chunk": v["frames_per_chunk"],
+                   "height": v["height"], "width": v["width"], "channels": v["channels"],
+                   "parallelism": "replica%d" % world,
+                   "l2": "no flush: per-chunk working set %.0f MB > 126 MB L2" % (
+                       8 * v["frames_per_chunk"] * v["height"] * v["width"] * v["channels"]
+                       * 2 / 1e6)},
+        "roofline": v["conv"], "vae_stage": v, "gpu_launches": 4 * args.steps,
+        "clocks": v["clocks"],
+    }
+
+
 def run_config_legs(args, dev, peaks):
     """The other configurations of the benchmark, each a short leg with its own
     clock record: the tiny wave (latency), the 5-step and 14B waves, the 30-layer
@@ -1515,7 +1547,10 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="wan13b_4step", choices=sorted(wi.WORKLOADS))
+    ap.add_argument("--workload", default="wan13b_4step",
+                    choices=sorted(wi.WORKLOADS) + ["vae_stage"],
+                    help="vae_stage: only the streaming VAE-decode stage (residual block of "
+                         "causal 3x3x3 convolutions at 120 x 208 x 384, 12 frames per chunk)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-block", action="store_true",
@@ -1535,6 +1570,16 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    if args.workload == "vae_stage":
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the reference arm times the "
+                              "attention oracle; vae_stage has no CPU reference leg"}))
+            return
+        rank, world, local = dist_setup(args.gpus)
+        line = run_vae(args, rank, world, local)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
     if args.attn != "bf16" and wi.WORKLOADS[args.workload].layers > 1:
         raise SystemExit("--attn %s times single-layer workloads only" % args.attn)
     rank, world, local = dist_setup(args.gpus)

@@ -575,38 +575,46 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
             }
         }
     } else if (warp == 1) {
-        if (lane == 0 && leader) {
+        if (leader) {
             // ---------------- MMA issuer (leader CTA, for the pair) ----------------
+            // The whole warp runs the loop and its waits (warp-uniform values), one
+            // elected lane issues the MMAs and commits (as in the attention kernel:
+            // a single divergent lane issues measurably fewer MMAs per cycle).
+            const bool issuer = elect_one_sync();
             constexpr uint32_t idesc = idesc_bf16_f32(2 * BM, BN, false);
             constexpr uint32_t hi = sw128_desc_hi(1024);
             uint32_t it = 0, acc_it = 0;
             bool ok = true;
             for (int t = cid; ok && t < p.n_tiles; t += ncl, ++acc_it) {
                 const uint32_t b = acc_it & 1u;
-                if (!(ok = wait_bar(bar(B::acc_empty + b), ((acc_it >> 1) & 1u) ^ 1u, ctl,
-                                    kWhereMmaAcc)))
-                    break;
+                ok = wait_bar(bar(B::acc_empty + b), ((acc_it >> 1) & 1u) ^ 1u, ctl, kWhereMmaAcc);
+                if (!(ok = __all_sync(0xFFFFFFFFu, ok))) break;
                 tc_fence_after();
                 const uint32_t d = tmem + b * BN;
                 for (int kb = 0; kb < nk; ++kb, ++it) {
                     const uint32_t st = it % kStages;
-                    if (!(ok = wait_bar(bar(B::full + st), (it / kStages) & 1u, ctl, kWhereMmaFull)))
-                        break;
+                    ok = wait_bar(bar(B::full + st), (it / kStages) & 1u, ctl, kWhereMmaFull);
+                    if (!(ok = __all_sync(0xFFFFFFFFu, ok))) break;
                     tc_fence_after();
-                    const uint32_t alo = sw128_desc_lo(sbase + st * kStageBytes, 16);
-                    const uint32_t blo = sw128_desc_lo(sbase + st * kStageBytes + kABytes, 16);
+                    if (issuer) {
+                        const uint32_t alo = sw128_desc_lo(sbase + st * kStageBytes, 16);
+                        const uint32_t blo = sw128_desc_lo(sbase + st * kStageBytes + kABytes, 16);
 #pragma unroll
-                    for (int s = 0; s < BK / 16; ++s)
-                        umma_ss_pair(d, desc_join(alo + ((s * 32) >> 4), hi),
-                                     desc_join(blo + ((s * 32) >> 4), hi), idesc,
-                                     (kb | s) ? 1u : 0u);
-                    umma_commit_pair_mc(bar(B::empty + st), 0x3);
+                        for (int s = 0; s < BK / 16; ++s)
+                            umma_ss_pair(d, desc_join(alo + ((s * 32) >> 4), hi),
+                                         desc_join(blo + ((s * 32) >> 4), hi), idesc,
+                                         (kb | s) ? 1u : 0u);
+                        umma_commit_pair_mc(bar(B::empty + st), 0x3);
+                    }
+                    __syncwarp();
                 }
                 if (!ok) break;
-                umma_commit_pair_mc(bar(B::acc_full + b), 0x3);
+                if (issuer) umma_commit_pair_mc(bar(B::acc_full + b), 0x3);
+                __syncwarp();
             }
             // every MMA of the pair completes before either CTA releases TMEM
-            umma_commit_pair_mc(bar(B::drain), 0x1);
+            if (issuer) umma_commit_pair_mc(bar(B::drain), 0x1);
+            __syncwarp();
             wait_bar(bar(B::drain), 0u, ctl, kWhereDrain, true);
         }
     } else {

@@ -7,9 +7,12 @@
 // (channels-last [pixels][C] bf16, gamma [C] fp32, fp32 arithmetic, one rounding
 // to bf16).
 //
-// HBM-bound (4 bytes per element).  One warp per pixel: lane l holds the
-// 8-channel pieces l, l + 32, ... of the row in registers between the sum of
-// squares and the output pass; gamma is read through the read-only path.
+// HBM-bound (4 bytes per element; the IEEE division of SiLU made it MUFU- and
+// issue-bound, 4.1 TB/s).  Half a warp per pixel: lane l of the half
+// holds the 8-channel pieces l, l + 16, ... of the row in registers between the
+// sum of squares and the output pass (3 pieces per lane at C = 384), so every
+// lane keeps several 16-byte loads in flight; gamma is read through the
+// read-only path.
 #include <cuda_bf16.h>
 
 #include "sm100.cuh"
@@ -20,23 +23,25 @@ namespace wf {
 namespace {
 
 constexpr int kWarps = 8;
+constexpr int kLanesPerRow = 16;
+constexpr int kRowsPerBlock = kWarps * 32 / kLanesPerRow;
 
-template <int PPL>    // 8-channel pieces per lane (C <= 256 * PPL)
+template <int PPL>    // 8-channel pieces per lane (C <= 8 * 16 * PPL)
 __global__ void __launch_bounds__(32 * kWarps) rms_norm_silu_kernel(const uint16_t *__restrict__ x,
                                                                     const float *__restrict__ gamma,
                                                                     uint16_t *__restrict__ y,
                                                                     long M, int C, float eps)
 {
-    const int lane = threadIdx.x & 31;
-    const long row = static_cast<long>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
-    if (row >= M) return;                          // whole warp
+    const int sub = threadIdx.x & (kLanesPerRow - 1);
+    const long row = static_cast<long>(blockIdx.x) * kRowsPerBlock + threadIdx.x / kLanesPerRow;
+    const bool live = row < M;            // both halves of a warp take part in the shuffles
     const int pieces = C / 8;
-    const uint4 *src = reinterpret_cast<const uint4 *>(x + row * C);
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + (live ? row : 0) * C);
     uint4 u[PPL];
 #pragma unroll
     for (int i = 0; i < PPL; ++i) {
-        const int pc = lane + 32 * i;
-        u[i] = pc < pieces ? __ldcs(src + pc) : make_uint4(0u, 0u, 0u, 0u);
+        const int pc = sub + kLanesPerRow * i;
+        u[i] = live && pc < pieces ? __ldcs(src + pc) : make_uint4(0u, 0u, 0u, 0u);
     }
     float ss = 0.0f;
 #pragma unroll
@@ -49,12 +54,13 @@ __global__ void __launch_bounds__(32 * kWarps) rms_norm_silu_kernel(const uint16
         }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+    for (int o = kLanesPerRow / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+    if (!live) return;
     const float r = rsqrtf(ss / static_cast<float>(C) + eps);
     uint4 *dst = reinterpret_cast<uint4 *>(y + row * C);
 #pragma unroll
     for (int i = 0; i < PPL; ++i) {
-        const int pc = lane + 32 * i;
+        const int pc = sub + kLanesPerRow * i;
         if (pc >= pieces) break;
         const float4 *g4 = reinterpret_cast<const float4 *>(gamma + 8 * pc);
         const float4 ga = __ldg(g4), gb = __ldg(g4 + 1);
@@ -65,8 +71,10 @@ __global__ void __launch_bounds__(32 * kWarps) rms_norm_silu_kernel(const uint16
         for (int e = 0; e < 4; ++e) {
             float a = __uint_as_float(w[e] << 16) * r * g[2 * e];
             float b = __uint_as_float(w[e] & 0xFFFF0000u) * r * g[2 * e + 1];
-            a = a / (1.0f + __expf(-a));           // SiLU; -inf exponent gives -0
-            b = b / (1.0f + __expf(-b));
+            // SiLU as y / (1 + e^-y) with the approximate exponential and division
+            // (two MUFU operations, ~2^-21 relative error); a huge e^-y gives -0
+            a = __fdividef(a, 1.0f + __expf(-a));
+            b = __fdividef(b, 1.0f + __expf(-b));
             o[e] = pack_bf16x2(a, b);
         }
         __stcs(dst + pc, make_uint4(o[0], o[1], o[2], o[3]));
@@ -75,17 +83,20 @@ __global__ void __launch_bounds__(32 * kWarps) rms_norm_silu_kernel(const uint16
 
 }  // namespace
 
-int rms_norm_silu_max_channels() { return 512; }
+int rms_norm_silu_max_channels() { return 8 * kLanesPerRow * 4; }
 
 cudaError_t launch_rms_norm_silu(const uint16_t *x, const float *gamma, uint16_t *y, long M, int C,
                                  float eps, cudaStream_t stream)
 {
     if (M == 0) return cudaSuccess;
-    const dim3 grid(static_cast<unsigned>((M + kWarps - 1) / kWarps));
-    if (C <= 256)
-        rms_norm_silu_kernel<1><<<grid, 32 * kWarps, 0, stream>>>(x, gamma, y, M, C, eps);
-    else
-        rms_norm_silu_kernel<2><<<grid, 32 * kWarps, 0, stream>>>(x, gamma, y, M, C, eps);
+    const dim3 grid(static_cast<unsigned>((M + kRowsPerBlock - 1) / kRowsPerBlock));
+    const int ppl = (C / 8 + kLanesPerRow - 1) / kLanesPerRow;
+    switch (ppl) {
+    case 1: rms_norm_silu_kernel<1><<<grid, 32 * kWarps, 0, stream>>>(x, gamma, y, M, C, eps); break;
+    case 2: rms_norm_silu_kernel<2><<<grid, 32 * kWarps, 0, stream>>>(x, gamma, y, M, C, eps); break;
+    case 3: rms_norm_silu_kernel<3><<<grid, 32 * kWarps, 0, stream>>>(x, gamma, y, M, C, eps); break;
+    default: rms_norm_silu_kernel<4><<<grid, 32 * kWarps, 0, stream>>>(x, gamma, y, M, C, eps); break;
+    }
     return cudaGetLastError();
 }
 
