@@ -74,10 +74,21 @@ constexpr unsigned long long kDrainLimit = 1ull << 32;
 // Shared-memory plan per epilogue: the stage ring, then (QKV only) the RoPE
 // (cos, sin) tables, the epilogue warps' staging buffers and the barrier block.
 // (Six stages measured 1-4% faster than seven; with the tables only five fit.)
+// A stage of a convolution holds the input box of 16 columns x 10 rows x 64
+// channels (the 8 output rows of this CTA and one row above and below) and the
+// weights of the three row taps dy = 0, 1, 2 of one (dt, dx): the MMAs of tap dy
+// read the box from its row 16 dy on (a 2 KB offset, a whole number of 1024-byte
+// swizzle atoms), so a box is loaded once per three taps instead of three times.
+constexpr int kConvBoxRows = 10;
+constexpr uint32_t kConvABytes = 16 * kConvBoxRows * BK * 2;   // 20 KB
+
 template <int Epi, int BN>
 struct Smem {
-    static constexpr uint32_t kStageBytes = Tile<BN>::kStageBytes;
-    static constexpr int kStages = Epi == kEpiQkvAppend ? 5 : (BN == 192 ? 7 : 6);
+    static constexpr bool kConv = IsConv<Epi>::value;
+    static constexpr uint32_t kStageBytes =
+        kConv ? kConvABytes + 3 * Tile<BN>::kBBytes : Tile<BN>::kStageBytes;
+    static constexpr int kStages =
+        kConv ? 3 : (Epi == kEpiQkvAppend ? 5 : (BN == 192 ? 7 : 6));
     static constexpr uint32_t kTabOff = kStages * kStageBytes;
     static constexpr uint32_t kStgOff = kTabOff + (Epi == kEpiQkvAppend ? kTabMax * 8 : 0);
     static constexpr uint32_t kBarOff = kStgOff + kEpiWarps * kWarpStageBytes;
@@ -436,7 +447,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
 {
     using B = Smem<Epi, BN>;
     constexpr int kStages = B::kStages;
-    constexpr uint32_t kStageBytes = Tile<BN>::kStageBytes;
+    constexpr uint32_t kStageBytes = B::kStageBytes;
+    constexpr uint32_t kBBytes = Tile<BN>::kBBytes;
     constexpr bool kConv = IsConv<Epi>::value;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -454,8 +466,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     const int cid = static_cast<int>(cluster_id_x());
     const int ncl = static_cast<int>(nclusters_x());
     auto lead = [&](int i) -> uint32_t { return map_to_rank(bar(i), 0); };
-    // K slices: one per 64 columns of K, or per (tap, 64 input channels) of a conv
-    const int nk = kConv ? 27 * p.n_cblk : (p.K + BK - 1) / BK;
+    // K stages: one per 64 columns of K, or per (dt, dx, 64 input channels) of a
+    // convolution (each stage covering the three row taps dy)
+    const int nk = kConv ? 9 * p.n_cblk : (p.K + BK - 1) / BK;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -544,18 +557,21 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                     if (leader) mbar_arrive_expect_tx(bar(B::full + st), 2 * kStageBytes);
                     const uint32_t dst = sbase + st * kStageBytes;
                     if constexpr (kConv) {
-                        // tap (dt, dy, dx), channels [64 cb, 64 cb + 64): A is the 16 x 8
-                        // pixel box shifted by the tap (rows and columns outside the frame
-                        // read zeros); taps before the chunk read the history's frame
-                        // tf + 2, or zeros at the start of the video
-                        const int tap = kb / p.n_cblk, cb = kb - tap * p.n_cblk;
-                        const int dt = tap / 9, dy = (tap / 3) % 3, dx = tap % 3;
+                        // taps (dt, 0..2, dx), channels [64 cb, 64 cb + 64): A is the 16 x 10
+                        // pixel box from row ya - 1, shifted by dx (rows and columns outside
+                        // the frame read zeros); taps before the chunk read the history's
+                        // frame tf + 2, or zeros at the start of the video
+                        const int tdx = kb / p.n_cblk, cb = kb - tdx * p.n_cblk;
+                        const int dt = tdx / 3, dx = tdx - 3 * dt;
                         const int tf = fr + dt - 2;
                         const bool hist = tf < 0 && p.use_hist;
                         tma_load_4d_pair(dst, hist ? &tmap_h : &tmap_a, lead(B::full + st),
-                                         cb * BK, xa + dx - 1, ya + dy - 1, hist ? tf + 2 : tf);
-                        tma_load_3d_pair(dst + kABytes, &tmap_b, lead(B::full + st), cb * BK, tap,
-                                         brow);
+                                         cb * BK, xa + dx - 1, ya - 1, hist ? tf + 2 : tf);
+#pragma unroll
+                        for (int dy = 0; dy < 3; ++dy)
+                            tma_load_3d_pair(dst + kConvABytes + dy * kBBytes, &tmap_b,
+                                             lead(B::full + st), cb * BK, dt * 9 + dy * 3 + dx,
+                                             brow);
                     } else {
                         tma_load_2d_pair(dst, &tmap_a, lead(B::full + st), kb * BK, arow);
                         tma_load_2d_pair(dst + kABytes, &tmap_b, lead(B::full + st), kb * BK,
@@ -597,13 +613,29 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                     if (!(ok = __all_sync(0xFFFFFFFFu, ok))) break;
                     tc_fence_after();
                     if (issuer) {
-                        const uint32_t alo = sw128_desc_lo(sbase + st * kStageBytes, 16);
-                        const uint32_t blo = sw128_desc_lo(sbase + st * kStageBytes + kABytes, 16);
+                        if constexpr (kConv) {
+                            const uint32_t a0 = sbase + st * kStageBytes;
 #pragma unroll
-                        for (int s = 0; s < BK / 16; ++s)
-                            umma_ss_pair(d, desc_join(alo + ((s * 32) >> 4), hi),
-                                         desc_join(blo + ((s * 32) >> 4), hi), idesc,
-                                         (kb | s) ? 1u : 0u);
+                            for (int dy = 0; dy < 3; ++dy) {
+                                const uint32_t alo = sw128_desc_lo(a0 + dy * 2048, 16);
+                                const uint32_t blo =
+                                    sw128_desc_lo(a0 + kConvABytes + dy * kBBytes, 16);
+#pragma unroll
+                                for (int s = 0; s < BK / 16; ++s)
+                                    umma_ss_pair(d, desc_join(alo + ((s * 32) >> 4), hi),
+                                                 desc_join(blo + ((s * 32) >> 4), hi), idesc,
+                                                 (kb | dy | s) ? 1u : 0u);
+                            }
+                        } else {
+                            const uint32_t alo = sw128_desc_lo(sbase + st * kStageBytes, 16);
+                            const uint32_t blo =
+                                sw128_desc_lo(sbase + st * kStageBytes + kABytes, 16);
+#pragma unroll
+                            for (int s = 0; s < BK / 16; ++s)
+                                umma_ss_pair(d, desc_join(alo + ((s * 32) >> 4), hi),
+                                             desc_join(blo + ((s * 32) >> 4), hi), idesc,
+                                             (kb | s) ? 1u : 0u);
+                        }
                         umma_commit_pair_mc(bar(B::empty + st), 0x3);
                     }
                     __syncwarp();
@@ -735,7 +767,7 @@ cudaError_t launch_gemm(const CUtensorMap &ma, const CUtensorMap &mb, const Gemm
 }
 
 // Causal 3x3x3 convolution as an implicit GEMM: mx over the chunk [ct][ch][cw][cin]
-// and mh over its two history frames (box 64 channels x 16 columns x 8 rows x 1
+// and mh over its two history frames (box 64 channels x 16 columns x 10 rows x 1
 // frame), mw over the weights [N][27][cin] (box 64 x 1 x BN / 2), 128-byte swizzle.
 // bn: the tile width the maps were encoded for (192 or 256).
 cudaError_t launch_conv(const CUtensorMap &mx, const CUtensorMap &mh, const CUtensorMap &mw,

@@ -158,8 +158,9 @@ bool encode_map_2d(CUtensorMap *map, const void *base, long rows, long cols)
 }
 
 // 4-D map over a channels-last video [T][H][W][C] bf16: box = 64 channels x 16
-// columns x 8 rows x 1 frame (128 pixels, one 128-byte swizzle row each); reads
-// outside the frame or before the first frame return zeros.
+// columns x 10 rows x 1 frame (160 pixels, one 128-byte swizzle row each: a CTA's
+// 8 output rows and the rows above and below); reads outside the frame or before
+// the first frame return zeros.
 bool encode_map_video(CUtensorMap *map, const void *base, int T, int H, int W, int C)
 {
     auto enc = wf::tensor_map_encoder();
@@ -168,7 +169,7 @@ bool encode_map_video(CUtensorMap *map, const void *base, int T, int H, int W, i
                                 static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
     const cuuint64_t pix = static_cast<cuuint64_t>(C) * 2;
     const cuuint64_t strides[3] = {pix, pix * W, pix * W * H};
-    const cuuint32_t box[4] = {64, 16, 8, 1};
+    const cuuint32_t box[4] = {64, 16, 10, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
