@@ -346,6 +346,18 @@ def run_ours(args, rank, world, local):
     torch.cuda.synchronize(dev)
     e2e_ms = allreduce_max(dist, s2.elapsed_time(t2), dev) / e2e_steps
     barrier(dist, dev)
+    # the PCIe floor of the end-to-end step: the same host bytes copied alone
+    # (pinned -> device, one copy per input tensor, CUDA events), best of 3
+    h2d_ms = []
+    for _ in range(3):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for src, dst in ((hq, q), (hk_, k), (hv_, v)):
+            dst.copy_(src, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        h2d_ms.append(a.elapsed_time(b))
+    h2d_gbs = 3 * tensor_bytes / (min(h2d_ms) * 1e-3) / 1e9
 
     clk = clocks.summary(t_wall0, t_wall1)
     block = None
@@ -447,6 +459,10 @@ def run_ours(args, rank, world, local):
             "ms_per_step": round(e2e_ms, 4),
             "h2d_bytes_per_step": 3 * tensor_bytes,
             "d2h_bytes_per_step": tensor_bytes,
+            # a step cannot be shorter than its host-to-device copy (the D2H of the
+            # previous round overlaps it on the other copy engine)
+            "h2d_gbs_measured": round(h2d_gbs, 2),
+            "pcie_floor_ms": round(3 * tensor_bytes / (h2d_gbs * 1e9) * 1e3, 4),
         },
         "gpu_launches": (3 if fp8 else 2) * args.steps,
         "clocks": clk,
