@@ -79,6 +79,29 @@ def run_all(wf):
     wf.wf_layer_norm_modulate(plan, xc, mod[0], mod[1], L, h)
     statuses["layer_norm"] = wf.wf_sync_status(plan)
     out["layer_norm"] = h.view(torch.int16).cpu().numpy()
+    # the fused-Q8 append, and the VAE stage's convolution (ragged frame, Cin not a
+    # multiple of 64, a partial output tile, history + residual) and RMSNorm + SiLU
+    q8b = torch.empty((T, H, D), dtype=torch.uint8, device=dev)
+    qsb = torch.empty((H, T), dtype=torch.float32, device=dev)
+    kc3, vc3 = kc.clone(), vc.clone()
+    wf.wf_qk_norm_rope_append_fp8q(plan, r, q, k, v, None, gq, gk, None, q8b, qsb, kc3, vc3)
+    statuses["append_q8"] = wf.wf_sync_status(plan)
+    out.update(append_q8=q8b.cpu().numpy(), append_qs=qsb.cpu().numpy())
+    Tv, Hv, Wv, Ci, Co = 3, 19, 21, 96, 160
+    xv = wi.bf16_normal((Tv, Hv, Wv, Ci), 10, wi.STREAM_X).to(dev)
+    hv = wi.bf16_normal((2, Hv, Wv, Ci), 10, wi.STREAM_CACHE).to(dev)
+    wv = wi.bf16_weight(Co, 27 * Ci, 10).reshape(Co, 3, 3, 3, Ci).contiguous().to(dev)
+    bv = wi.f32_vector((Co,), 0.1, 10, wi.STREAM_BIAS).to(dev)
+    rv = wi.bf16_normal((Tv, Hv, Wv, Co), 10, wi.STREAM_MOD).to(dev)
+    yv = torch.empty((Tv, Hv, Wv, Co), dtype=torch.bfloat16, device=dev)
+    wf.wf_causal_conv3d(plan, xv, hv, wv, bv, rv, yv)
+    statuses["conv"] = wf.wf_sync_status(plan)
+    out["conv"] = yv.view(torch.int16).cpu().numpy()
+    gv = (1 + wi.f32_vector((Ci,), 0.1, 10, wi.STREAM_GAMMA)).to(dev)
+    nv = torch.empty_like(xv)
+    wf.wf_rms_norm_silu(plan, xv, gv, nv)
+    statuses["rms_norm_silu"] = wf.wf_sync_status(plan)
+    out["rms_norm_silu"] = nv.view(torch.int16).cpu().numpy()
     plan.destroy()
     return out, statuses
 
