@@ -9,9 +9,14 @@
 // masked tiles are never loaded, and the only element mask is "key row < L" in
 // the last 128-key tile of each chunk (TMA fills the rows past L with zeros).
 //
-// Work unit = (wave chunk c, head h, pair of 128-row query tiles).  Units are
-// numbered longest first (cost (h_valid + c + 1) key chunks); one CTA per SM
-// pops them from a global counter (greedy longest-processing-time order).
+// Work unit = (wave chunk c, head h, pair of 128-row query tiles).  One CTA per
+// SM pops units from a global counter.  The heads are taken in blocks of
+// head_block (chosen on the host): all units of one block, longest first (cost
+// (h_valid + c + 1) key chunks; greedy longest-processing-time order inside the
+// block), then the next block.  The units of a block read the same key/value
+// chunks of its heads at nearly the same time, and the host keeps a block's
+// keys and values within half of L2, so a key tile comes from DRAM about once
+// instead of once for every wave chunk that sees it.
 // Warp roles (384 threads, three warpgroups):
 //   warps 0-3   softmax for query tile 0 (TMEM lanes 0..127, one row per thread)
 //   warps 4-7   softmax for query tile 1
@@ -137,12 +142,20 @@ struct Unit {
 __device__ __forceinline__ Unit decode_unit(const AttnParams &p, int u)
 {
     Unit r;
-    const int per_c = p.H * p.n_qpairs;
-    const int ci = u / per_c;
-    const int rem = u - ci * per_c;
-    r.c = p.W - 1 - ci;                       // longest (latest chunk) first
-    r.h = rem / p.n_qpairs;
-    r.pair = rem - r.h * p.n_qpairs;
+    // blocks of head_block heads, one after the other (the last may hold fewer);
+    // inside a block the latest chunk's units (the longest) first, then by head
+    // and query tile pair
+    const int blk_units = p.head_block * p.W * p.n_qpairs;
+    const int hb = u / blk_units;
+    const int rem_b = u - hb * blk_units;
+    const int gb = min(p.head_block, p.H - hb * p.head_block);
+    const int per_c = gb * p.n_qpairs;
+    const int ci = rem_b / per_c;
+    const int rem = rem_b - ci * per_c;
+    const int hi = rem / p.n_qpairs;
+    r.c = p.W - 1 - ci;
+    r.h = hb * p.head_block + hi;
+    r.pair = rem - hi * p.n_qpairs;
     r.n_kt = (p.h_valid + r.c + 1) * p.n_ktiles;
     r.has1 = (2 * r.pair + 1) * BM < p.L;
     return r;

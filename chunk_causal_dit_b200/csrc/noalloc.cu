@@ -124,9 +124,10 @@ extern "C" int wf_chunk_causal_attn_noalloc(int chunk_tokens, int n_wave_chunks,
         (reinterpret_cast<uintptr_t>(lse) & 3u))
         return WF_ERR_INVALID_ARG;
 
-    int dev = -1, sms = 0, ma = 0, mi = 0;
+    int dev = -1, sms = 0, ma = 0, mi = 0, l2 = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&ma, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&mi, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
         (void)cudaGetLastError();
@@ -155,6 +156,9 @@ extern "C" int wf_chunk_causal_attn_noalloc(int chunk_tokens, int n_wave_chunks,
     a.n_ktiles = n_ktiles;
     a.n_qpairs = n_qpairs;
     a.n_units = heads * n_wave_chunks * n_qpairs;
+    const int grid = a.n_units < sms ? a.n_units : sms;
+    a.head_block = wf::attn_head_block(heads, n_wave_chunks, a.h_valid, chunk_tokens, head_dim, 2,
+                                       l2, grid);
     a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(head_dim)));
     a.wait_limit = 1ull << 32;
     a.withhold_q = 0;
@@ -167,6 +171,5 @@ extern "C" int wf_chunk_causal_attn_noalloc(int chunk_tokens, int n_wave_chunks,
     // status and timeout site start at zero for this call (the work counter is
     // cleared by the launch itself)
     if (cudaMemsetAsync(scratch, 0, 2 * sizeof(uint32_t), st) != cudaSuccess) return WF_ERR_CUDA;
-    const int grid = a.n_units < sms ? a.n_units : sms;
     return wf::launch_attn(mq, mk, mv, a, head_dim, grid, st) == cudaSuccess ? WF_OK : WF_ERR_CUDA;
 }

@@ -99,6 +99,71 @@ int check_round_shape(int chunk_tokens, int n_wave_chunks, int n_hist_chunks, in
     return WF_OK;
 }
 
+// Heads per block of the attention's unit order.  The units of a block of heads
+// are handed out before the next block's, longest first inside the block, so
+// the keys and values being read at any moment are those of one or two blocks.
+// A block's visible key/value chunks (h_valid + W of them, for each of its
+// heads) are kept within half of the L2 cache, so that every unit that reads
+// a key tile after the first finds it in L2.  Among the counts that fit, the
+// one whose schedule ends earliest is taken: each count is played through the
+// kernel's dynamic schedule (each unit goes to the CTA that frees first; a
+// unit costs its key tiles, 0.93 of that for a one-tile unit, plus 3 tiles of
+// set-up), with ties going to the larger count.  Results do not depend on it:
+// every unit computes the same rows in the same order.
+int attn_head_block(int H, int W, int h_valid, int L, int D, int k_bytes, long long l2_bytes,
+                    int n_ctas)
+{
+    const double per_head = static_cast<double>(h_valid + W) * L * D * (k_bytes + 2);
+    long long g_max = H;
+    if (l2_bytes > 0) {
+        g_max = static_cast<long long>(0.5 * static_cast<double>(l2_bytes) / per_head);
+        g_max = g_max < 1 ? 1 : (g_max > H ? H : g_max);
+    }
+    const int n_ktiles = (L + 127) / 128;
+    const int n_qpairs = (n_ktiles + 1) / 2;
+    const long long n_units = static_cast<long long>(H) * W * n_qpairs;
+    constexpr int kMaxCtas = 1024;
+    if (n_ctas < 1 || n_ctas > kMaxCtas || n_units * g_max > (4ll << 20))
+        return static_cast<int>(g_max);
+    double t[kMaxCtas];
+    int best_g = static_cast<int>(g_max);
+    double best = 0.0;
+    for (int g = static_cast<int>(g_max); g >= 1; --g) {
+        for (int i = 0; i < n_ctas; ++i) t[i] = 0.0;
+        for (int hb = 0; hb < H; hb += g) {
+            const int gb = H - hb < g ? H - hb : g;
+            for (int c = W - 1; c >= 0; --c)
+                for (int k = 0; k < gb * n_qpairs; ++k) {
+                    const int pair = k % n_qpairs;
+                    const bool has1 = (2 * pair + 1) * 128 < L;
+                    const double d =
+                        static_cast<double>(h_valid + c + 1) * n_ktiles * (has1 ? 1.0 : 0.93) + 3.0;
+                    // the CTA that frees first (heap root) takes the unit
+                    double v = t[0] + d;
+                    int i = 0;
+                    while (true) {
+                        const int l = 2 * i + 1, r = l + 1;
+                        int m = i;
+                        double mv = v;
+                        if (l < n_ctas && t[l] < mv) { m = l; mv = t[l]; }
+                        if (r < n_ctas && t[r] < mv) { m = r; mv = t[r]; }
+                        if (m == i) break;
+                        t[i] = t[m];
+                        i = m;
+                    }
+                    t[i] = v;
+                }
+        }
+        double end = 0.0;
+        for (int i = 0; i < n_ctas; ++i) end = t[i] > end ? t[i] : end;
+        if (g == g_max || end < best * (1.0 - 2e-3)) {
+            best = end;
+            best_g = g;
+        }
+    }
+    return best_g;
+}
+
 }  // namespace wf
 
 namespace {
@@ -244,20 +309,25 @@ int wf_plan(int chunk_tokens, int n_wave_chunks, int n_hist_chunks, int heads, i
     p->attn_kernel = WF_ATTN_AUTO;
     p->device = -1;
     p->num_sms = 0;
+    p->l2_bytes = 0;
+    p->head_block = 0;
+    std::memset(p->head_block_cache, 0, sizeof(p->head_block_cache));
     p->cc_major = p->cc_minor = 0;
     p->words = nullptr;
 
     int dev = -1;
     if (cudaGetDevice(&dev) == cudaSuccess) {
-        int sms = 0, ma = 0, mi = 0;
+        int sms = 0, ma = 0, mi = 0, l2 = 0;
         void *w = nullptr;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) == cudaSuccess &&
             cudaDeviceGetAttribute(&ma, cudaDevAttrComputeCapabilityMajor, dev) == cudaSuccess &&
             cudaDeviceGetAttribute(&mi, cudaDevAttrComputeCapabilityMinor, dev) == cudaSuccess &&
             cudaMalloc(&w, sizeof(wf::DeviceWords)) == cudaSuccess) {
             if (cudaMemset(w, 0, sizeof(wf::DeviceWords)) == cudaSuccess) {
                 p->device = dev;
                 p->num_sms = sms;
+                p->l2_bytes = l2;
                 p->cc_major = ma;
                 p->cc_minor = mi;
                 p->words = static_cast<wf::DeviceWords *>(w);
@@ -325,6 +395,49 @@ int wf_plan_set_attn_kernel(wf_plan_t p, int kind)
     if (kind == WF_ATTN_PAIR && p->D != 128) return WF_ERR_UNSUPPORTED;
     p->attn_kernel = kind;
     return WF_OK;
+}
+
+int wf_plan_set_head_block(wf_plan_t p, int heads)
+{
+    if (p == nullptr || heads < 0 || heads > p->H) return WF_ERR_INVALID_ARG;
+    p->head_block = heads;
+    return WF_OK;
+}
+
+namespace {
+
+// The attention's heads per block for a round with h_valid history chunks: the
+// plan's setting, else wf::attn_head_block's choice (kept per h_valid).
+int plan_head_block(wf_plan_s *p, int h_valid, bool fp8_keys, int grid)
+{
+    if (p->head_block > 0) return p->head_block;
+    int *slot = h_valid < 8 ? &p->head_block_cache[fp8_keys ? 1 : 0][h_valid] : nullptr;
+    if (slot != nullptr && *slot > 0) return *slot;
+    const int g = wf::attn_head_block(p->H, p->W, h_valid, p->L, p->D, fp8_keys ? 1 : 2,
+                                      p->l2_bytes, grid);
+    if (slot != nullptr) *slot = g;
+    return g;
+}
+
+}  // namespace
+
+int wf_plan_head_block(wf_plan_t p, long round, int fp8_keys)
+{
+    if (p == nullptr || round < 0) return -1;
+    const int n_qpairs = ((p->L + 127) / 128 + 1) / 2;
+    const int n_units = p->H * p->W * n_qpairs;
+    const int grid = n_units < p->num_sms ? n_units : p->num_sms;
+    return plan_head_block(p, wf::history_valid(round, p->Hh), fp8_keys != 0, grid);
+}
+
+int wf_attn_head_block(int heads, int n_wave_chunks, int h_valid, int chunk_tokens, int head_dim,
+                       int key_bytes, long long l2_bytes, int n_ctas)
+{
+    if (heads < 1 || n_wave_chunks < 1 || h_valid < 0 || chunk_tokens < 1 || head_dim < 1 ||
+        (key_bytes != 1 && key_bytes != 2))
+        return -1;
+    return wf::attn_head_block(heads, n_wave_chunks, h_valid, chunk_tokens, head_dim, key_bytes,
+                               l2_bytes, n_ctas);
 }
 
 void wf_plan_destroy(wf_plan_t p)
@@ -447,6 +560,8 @@ int wf_chunk_causal_attn(wf_plan_t p, long round, const void *q_out, const void 
     a.n_ktiles = (p->L + 127) / 128;
     a.n_qpairs = (a.n_ktiles + 1) / 2;
     a.n_units = p->H * p->W * a.n_qpairs;
+    a.head_block = plan_head_block(p, a.h_valid, false,
+                                   a.n_units < p->num_sms ? a.n_units : p->num_sms);
     a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(p->D)));
     a.wait_limit = p->wait_limit;
     a.withhold_q = p->withhold_q;
@@ -526,6 +641,8 @@ int wf_chunk_causal_attn_fp8qk(wf_plan_t p, long round, const void *q8, const fl
     a.n_ktiles = (p->L + 127) / 128;
     a.n_qpairs = (a.n_ktiles + 1) / 2;
     a.n_units = p->H * p->W * a.n_qpairs;
+    a.head_block = plan_head_block(p, a.h_valid, true,
+                                   a.n_units < p->num_sms ? a.n_units : p->num_sms);
     a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(p->D)));
     a.wait_limit = p->wait_limit;
     a.withhold_q = p->withhold_q;

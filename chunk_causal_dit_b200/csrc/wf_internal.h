@@ -78,6 +78,7 @@ struct AttnParams {
     int n_qpairs;             // query tile pairs per chunk: ceil(ceil(L/128)/2)
     int n_ktiles;             // key tiles per chunk: ceil(L/128)
     int n_units;              // H * W * n_qpairs
+    int head_block;           // heads per block of the unit order (1..H)
     float scale_log2;         // log2(e) / sqrt(D)
     unsigned long long wait_limit;  // SM clock cycles
     int withhold_q;           // test hook: withhold each CTA's first Q-tile copy
@@ -144,6 +145,11 @@ bool encode_map(CUtensorMap *map, const void *base, int D, int H, int n2, int n2
 // WF_OK, or the status wf_plan returns for this shape.
 int check_round_shape(int chunk_tokens, int n_wave_chunks, int n_hist_chunks, int heads,
                       int head_dim);
+// Heads per block of the attention's unit order (1..H) for a round with h_valid
+// history chunks; k_bytes is the size of a key element (2 bf16, 1 E4M3),
+// l2_bytes the device's L2 size, n_ctas the attention grid.
+int attn_head_block(int H, int W, int h_valid, int L, int D, int k_bytes, long long l2_bytes,
+                    int n_ctas);
 
 }  // namespace wf
 
@@ -157,6 +163,9 @@ struct wf_plan_s {
     int attn_kernel;          // WF_ATTN_* (wf_plan_set_attn_kernel)
     int device;               // -1: no device state
     int num_sms;
+    long long l2_bytes;       // L2 cache size of `device`
+    int head_block;           // attention unit order: heads per block, 0 = chosen per round
+    int head_block_cache[2][8];   // attention head blocks by [fp8 keys][h_valid], 0: not yet
     int cc_major, cc_minor;   // compute capability of `device`
     wf::DeviceWords *words;   // device memory
 };

@@ -46,6 +46,9 @@ SIGNATURES = {
     "wf_plan_set_wait_limit": (_I, [_P, ctypes.c_ulonglong]),
     "wf_plan_set_withhold_q": (_I, [_P, _I]),
     "wf_plan_set_attn_kernel": (_I, [_P, _I]),
+    "wf_plan_set_head_block": (_I, [_P, _I]),
+    "wf_plan_head_block": (_I, [_P, _L, _I]),
+    "wf_attn_head_block": (_I, [_I, _I, _I, _I, _I, _I, ctypes.c_longlong, _I]),
     "wf_plan_destroy": (None, [_P]),
     "wf_cache_bytes": (ctypes.c_size_t, [_P]),
     "wf_useful_flops": (ctypes.c_double, [_P, _L]),
@@ -165,6 +168,15 @@ class Plan:
         _check(load().wf_plan_set_attn_kernel(self.handle, int(kind)), "wf_plan_set_attn_kernel")
         return self
 
+    def set_head_block(self, heads: int):
+        """Heads per block of the attention's unit order; 0 = chosen per call (see wf.h)."""
+        _check(load().wf_plan_set_head_block(self.handle, int(heads)), "wf_plan_set_head_block")
+        return self
+
+    def head_block(self, round_: int, fp8_keys: bool = False) -> int:
+        """Heads per block that round `round_`'s attention call uses."""
+        return int(load().wf_plan_head_block(self.handle, round_, int(bool(fp8_keys))))
+
     def destroy(self):
         if self.handle:
             load().wf_plan_destroy(self.handle)
@@ -185,6 +197,12 @@ class Plan:
 
 def wf_plan(chunk_tokens, n_wave_chunks, n_hist_chunks, heads, head_dim) -> Plan:
     return Plan(chunk_tokens, n_wave_chunks, n_hist_chunks, heads, head_dim)
+
+
+def wf_attn_head_block(heads, n_wave_chunks, h_valid, chunk_tokens, head_dim, key_bytes,
+                       l2_bytes, n_ctas) -> int:
+    return int(load().wf_attn_head_block(heads, n_wave_chunks, h_valid, chunk_tokens, head_dim,
+                                         key_bytes, l2_bytes, n_ctas))
 
 
 def wf_cache_bytes(plan: Plan) -> int:

@@ -126,6 +126,39 @@ WF_API int wf_plan_set_withhold_q(wf_plan_t plan, int on);
 #define WF_ATTN_PAIR 2
 WF_API int wf_plan_set_attn_kernel(wf_plan_t plan, int kind);
 
+/* Order of the attention's work units (single-CTA kernel, bf16 and FP8 Q.K^T).
+ * A unit is (wave chunk c, head h, pair of 128-row query tiles); it reads the
+ * key/value chunks that chunk-wise causal attention ("Wave Forcing", abstract)
+ * lets chunk c see: the valid history chunks and wave chunks 0..c of head h.
+ * The same key chunk is read by the units of every wave chunk at or after it,
+ * so the kernel takes the heads in blocks: all units of one block of heads,
+ * longest first inside the block, then the next block.
+ *
+ * wf_plan_set_head_block sets the heads per block, 1..heads; 0 (the default)
+ * lets each call choose with wf_attn_head_block.  Outputs are bit-identical
+ * for every value: each unit computes the same rows in the same order, only
+ * the order of the units changes.  WF_ERR_INVALID_ARG outside 0..heads or for
+ * a NULL plan. */
+WF_API int wf_plan_set_head_block(wf_plan_t plan, int heads);
+
+/* Heads per block that round `round`'s attention call uses (fp8_keys != 0: the
+ * FP8 Q.K^T call, whose keys are 1 byte).  -1 for a NULL plan or round < 0. */
+WF_API int wf_plan_head_block(wf_plan_t plan, long round, int fp8_keys);
+
+/* The choice itself (host arithmetic only).  A block's visible keys and values,
+ * (h_valid + n_wave_chunks) * chunk_tokens * head_dim * (key_bytes + 2) bytes
+ * per head, are kept within half of l2_bytes, so that the units reading a key
+ * tile after the first find it in L2; that caps the count at g_max (at least
+ * 1, at most heads; heads when l2_bytes <= 0).  Among 1..g_max the count whose
+ * schedule ends first is returned, each count played through the kernel's
+ * dynamic schedule over n_ctas CTAs (a unit costs its key tiles, 0.93 of that
+ * with a single query tile, plus 3 tiles of set-up; ties go to the larger
+ * count).  g_max is returned without that comparison when n_ctas is outside
+ * 1..1024 or the comparison would take over 4M unit steps.  Returns -1 for
+ * sizes that are not positive (h_valid < 0, key_bytes not 1 or 2). */
+WF_API int wf_attn_head_block(int heads, int n_wave_chunks, int h_valid, int chunk_tokens,
+                              int head_dim, int key_bytes, long long l2_bytes, int n_ctas);
+
 WF_API void wf_plan_destroy(wf_plan_t plan);
 
 /* Bytes of ONE ring (K or V): R * L * H * D * 2.  0 for a NULL plan. */

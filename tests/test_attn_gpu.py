@@ -204,6 +204,66 @@ def test_repeat_runs_bit_identical(wf, kernel):
     plan.destroy()
 
 
+@pytest.mark.parametrize("L,W,Hh,H,D,r", [(300, 3, 2, 7, 128, 4), (200, 3, 1, 5, 64, 3)])
+def test_head_blocks_all_rows(wf, L, W, Hh, H, D, r):
+    """Every head-block order of the work units gives bit-identical outputs
+    (each unit computes the same rows in the same order), and they match the
+    oracle on every row."""
+    q, kc, vc = place_round(L, W, Hh, H, D, r, seed=31 + D)
+    plan = wf.Plan(L, W, Hh, H, D)
+    outs = {}
+    for g in (H, 1, 2, 3, 0):
+        plan.set_head_block(g)
+        assert plan.head_block(r) == g if g else 1 <= plan.head_block(r) <= H
+        o = torch.full_like(q, float("nan"))
+        lse = torch.full((H, W * L), float("nan"), dtype=torch.float32, device=q.device)
+        wf.wf_chunk_causal_attn(plan, r, q, kc, vc, o, lse)
+        torch.cuda.synchronize()
+        assert wf.wf_sync_status(plan) == wf.WF_OK
+        outs[g] = (o, lse)
+    o0, lse0 = outs[H]
+    for g, (o, lse) in outs.items():
+        assert torch.equal(o.view(torch.int16), o0.view(torch.int16)), "head block %d" % g
+        assert torch.equal(lse, lse0), "head block %d" % g
+    cache = oracle_cache_from_ring(kc, vc, r, W, Hh)
+    T = W * L
+    rows = np.repeat(np.arange(T), H)
+    heads = np.tile(np.arange(H), T)
+    o_ref, lse_ref = oracle.round_attention(cache, r, W, Hh, wi.bits(q.cpu()), rows, heads)
+    o_gpu = outs[2][0].float().cpu().numpy().reshape(T * H, D)
+    assert_attention_close(o_gpu, o_ref, "head blocks L=%d H=%d D=%d" % (L, H, D))
+    assert np.max(np.abs(outs[2][1].cpu().numpy().T.reshape(-1) - lse_ref)) <= 1e-3
+    plan.destroy()
+
+
+def test_head_blocks_more_units_than_ctas(wf):
+    """A round with more work units than SMs, so that CTAs take several units
+    and the blocks follow one another through the global counter: every
+    head-block order gives the same bits, and no row is left unwritten."""
+    L, W, Hh, H, D, r = 1000, 4, 2, 12, 128, 3
+    q, kc, vc = place_round(L, W, Hh, H, D, r, seed=77)
+    plan = wf.Plan(L, W, Hh, H, D)
+    ref = None
+    for g in (H, 1, 2, 3, 5, 0):
+        plan.set_head_block(g)
+        o = torch.full_like(q, float("nan"))
+        wf.wf_chunk_causal_attn(plan, r, q, kc, vc, o, None)
+        torch.cuda.synchronize()
+        assert wf.wf_sync_status(plan) == wf.WF_OK
+        assert not torch.isnan(o).any(), "head block %d left rows unwritten" % g
+        if ref is None:
+            ref = o
+        assert torch.equal(o.view(torch.int16), ref.view(torch.int16)), "head block %d" % g
+    # sampled rows of the last chunk (the longest units) against the oracle
+    cache = oracle_cache_from_ring(kc, vc, r, W, Hh)
+    rows = np.repeat(np.array([(W - 1) * L, (W - 1) * L + 511, W * L - 1]), H)
+    heads = np.tile(np.arange(H), 3)
+    o_ref, _ = oracle.round_attention(cache, r, W, Hh, wi.bits(q.cpu()), rows, heads)
+    got = ref.float().cpu().numpy()[rows, heads]
+    assert_attention_close(got, o_ref, "head blocks, sampled rows")
+    plan.destroy()
+
+
 def test_ring_over_rounds_end_to_end(wf):
     # append + attention for rounds 0 .. 2R+1 against the oracle's absolute-id cache
     w = wi.Workload("ring", H=2, D=64, F=1, gh=5, gw=8, n_wave=3, n_hist=2)

@@ -143,6 +143,13 @@ def test_fp8qk_repeat_bit_identical_and_head_dim_64_unsupported(wf):
         wf.wf_chunk_causal_attn_fp8qk(plan, r, q8, qs, k8, ks, vc, o1)
         torch.cuda.synchronize()
         assert torch.equal(o0.view(torch.int16), o1.view(torch.int16))
+    # every head-block order of the units gives the same bits
+    for g in (1, 3, H):
+        plan.set_head_block(g)
+        o1.fill_(float("nan"))
+        wf.wf_chunk_causal_attn_fp8qk(plan, r, q8, qs, k8, ks, vc, o1)
+        torch.cuda.synchronize()
+        assert torch.equal(o0.view(torch.int16), o1.view(torch.int16)), "head block %d" % g
     plan.destroy()
     p64 = wf.Plan(200, 3, 1, 2, 64)
     with pytest.raises(wf.WFError) as e:
