@@ -211,7 +211,9 @@ def test_qkv_equals_projection_then_append(wf):
     plan.destroy()
 
 
-@pytest.mark.parametrize("M,C,rpg", [(1000, 1536, 300), (37, 5120, 10), (64, 8, 64), (5, 6144, 2)])
+@pytest.mark.parametrize("M,C,rpg", [(1000, 1536, 300), (37, 5120, 10), (64, 8, 64), (5, 6144, 2),
+                                     (1000, 2048, 7), (3, 1536, 1), (333, 2056, 50),
+                                     (4679, 1024, 4680), (23400, 1536, 4680)])
 def test_layer_norm_modulate_parity(wf, M, C, rpg):
     dev = "cuda"
     seed = M + C
