@@ -102,6 +102,27 @@ int scratch_for_current_device(int dev, void **out)
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Heads per block of the attention's unit order for the last shape seen on each
+// device.  The choice plays the kernel's schedule through on the host (tens to
+// hundreds of microseconds at model sizes), and a serving loop repeats one shape.
+struct HeadBlockEntry {
+    int H, W, h_valid, L, D, l2, grid, g;
+};
+std::mutex g_head_block_mu;
+HeadBlockEntry g_head_block[kMaxDevices] = {};
+
+int head_block_for(int dev, int H, int W, int h_valid, int L, int D, int l2, int grid)
+{
+    std::lock_guard<std::mutex> lock(g_head_block_mu);
+    HeadBlockEntry &e = g_head_block[dev];
+    if (e.g > 0 && e.H == H && e.W == W && e.h_valid == h_valid && e.L == L && e.D == D &&
+        e.l2 == l2 && e.grid == grid)
+        return e.g;
+    const int g = wf::attn_head_block(H, W, h_valid, L, D, 2, l2, grid);
+    e = HeadBlockEntry{H, W, h_valid, L, D, l2, grid, g};
+    return g;
+}
+
 }  // namespace
 
 extern "C" int wf_chunk_causal_attn_noalloc(int chunk_tokens, int n_wave_chunks,
@@ -157,8 +178,8 @@ extern "C" int wf_chunk_causal_attn_noalloc(int chunk_tokens, int n_wave_chunks,
     a.n_qpairs = n_qpairs;
     a.n_units = heads * n_wave_chunks * n_qpairs;
     const int grid = a.n_units < sms ? a.n_units : sms;
-    a.head_block = wf::attn_head_block(heads, n_wave_chunks, a.h_valid, chunk_tokens, head_dim, 2,
-                                       l2, grid);
+    a.head_block = head_block_for(dev, heads, n_wave_chunks, a.h_valid, chunk_tokens, head_dim, l2,
+                                  grid);
     a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(head_dim)));
     a.wait_limit = 1ull << 32;
     a.withhold_q = 0;
