@@ -2,6 +2,7 @@
 // validation, TMA tensor-map set-up, and the two hot-path launches.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <climits>
 #include <cmath>
 #include <cstring>
@@ -311,7 +312,12 @@ int wf_plan(int chunk_tokens, int n_wave_chunks, int n_hist_chunks, int heads, i
     p->num_sms = 0;
     p->l2_bytes = 0;
     p->head_block = 0;
-    std::memset(p->head_block_cache, 0, sizeof(p->head_block_cache));
+    try {   // h_valid = 0 .. min(Hh, 63) are kept; a longer history is rare
+        p->head_block_cache.assign(2 * static_cast<size_t>(std::min(n_hist_chunks, 63) + 1), 0);
+    } catch (...) {
+        delete p;
+        return WF_ERR_CUDA;
+    }
     p->cc_major = p->cc_minor = 0;
     p->words = nullptr;
 
@@ -411,12 +417,15 @@ namespace {
 int plan_head_block(wf_plan_s *p, int h_valid, bool fp8_keys, int grid)
 {
     if (p->head_block > 0) return p->head_block;
-    int *slot = h_valid < 8 ? &p->head_block_cache[fp8_keys ? 1 : 0][h_valid] : nullptr;
-    if (slot != nullptr && *slot > 0) return *slot;
-    const int g = wf::attn_head_block(p->H, p->W, h_valid, p->L, p->D, fp8_keys ? 1 : 2,
-                                      p->l2_bytes, grid);
-    if (slot != nullptr) *slot = g;
-    return g;
+    const int per_key = static_cast<int>(p->head_block_cache.size() / 2);
+    if (h_valid >= per_key)
+        return wf::attn_head_block(p->H, p->W, h_valid, p->L, p->D, fp8_keys ? 1 : 2,
+                                   p->l2_bytes, grid);
+    int &slot = p->head_block_cache[(fp8_keys ? 1 : 0) * per_key + h_valid];
+    if (slot <= 0)
+        slot = wf::attn_head_block(p->H, p->W, h_valid, p->L, p->D, fp8_keys ? 1 : 2, p->l2_bytes,
+                                   grid);
+    return slot;
 }
 
 }  // namespace

@@ -3,6 +3,7 @@
 // kernels, so that what the debug dump reports is what the kernels execute.
 #pragma once
 #include <cstdint>
+#include <vector>
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <nvtx3/nvToolsExt.h>
@@ -165,7 +166,7 @@ struct wf_plan_s {
     int num_sms;
     long long l2_bytes;       // L2 cache size of `device`
     int head_block;           // attention unit order: heads per block, 0 = chosen per round
-    int head_block_cache[2][8];   // attention head blocks by [fp8 keys][h_valid], 0: not yet
+    std::vector<int> head_block_cache;   // attention head blocks, [fp8 keys][h_valid 0..min(Hh, 63)]; 0: not yet
     int cc_major, cc_minor;   // compute capability of `device`
     wf::DeviceWords *words;   // device memory
 };
