@@ -161,6 +161,16 @@ __device__ __forceinline__ Unit decode_unit(const AttnParams &p, int u)
     return r;
 }
 
+// Advance (key tile, ring slot) by one key tile: the next chunk's tile 0 after
+// a chunk's last tile, in the next slot (visible chunks have consecutive ids).
+__device__ __forceinline__ void next_key_tile(int &t, int &slot, const AttnParams &p)
+{
+    if (++t == p.n_ktiles) {
+        t = 0;
+        slot = slot + 1 == p.R ? 0 : slot + 1;
+    }
+}
+
 // The descriptors of one operand tile differ only in the start-address field
 // (low 14 bits), so they are built from a 32-bit low word and a constant high
 // word: fewer live 64-bit values in the MMA-issuing thread.
@@ -326,10 +336,10 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                         }
                     }
                 }
-                for (int j = 0; ok && j < un.n_kt; ++j) {
-                    const int b = j / p.n_ktiles;
-                    const int t = j - b * p.n_ktiles;
-                    const int slot = ring_slot(visible_chunk_id(p.round, p.h_valid, b), p.R);
+                // key tile t of the visible chunk in ring slot `slot`: the visible
+                // chunks have consecutive ids, so their slots follow each other mod R
+                int t = 0, slot = ring_slot(visible_chunk_id(p.round, p.h_valid, 0), p.R);
+                for (int j = 0; ok && j < un.n_kt; ++j, next_key_tile(t, slot, p)) {
                     for (int kv = 0; kv < 2; ++kv) {
                         if (!(ok = wait_bar(bar(B::kv_empty + stage), kv_phase ^ 1u, ctl,
                                             kWhereProducerKV)))
@@ -497,13 +507,12 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 if (q_row < p.L) sq = p.q_scale[static_cast<long>(un.h) * p.T +
                                                 static_cast<long>(un.c) * p.L + q_row];
             float m_run = -INFINITY, l_run = 0.f;
-            int t = 0;                              // key tile inside its chunk
-            for (int j = 0; j < un.n_kt; ++j, t = (t + 1 == p.n_ktiles) ? 0 : t + 1) {
+            // key tile t inside its chunk, held in ring slot `slot`
+            int t = 0, slot = ring_slot(visible_chunk_id(p.round, p.h_valid, 0), p.R);
+            for (int j = 0; j < un.n_kt; ++j, next_key_tile(t, slot, p)) {
                 float scale = scale0;
                 if constexpr (F8) {
                     // s = (q8 . k8) * sq * sk: fold both scales into the exponent scale
-                    const int b = j / p.n_ktiles;
-                    const int slot = ring_slot(visible_chunk_id(p.round, p.h_valid, b), p.R);
                     scale = scale0 * sq *
                             p.k_scale[(static_cast<long>(slot) * p.n_ktiles + t) * p.H + un.h];
                 }
