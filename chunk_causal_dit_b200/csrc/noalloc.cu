@@ -194,3 +194,22 @@ extern "C" int wf_chunk_causal_attn_noalloc(int chunk_tokens, int n_wave_chunks,
     if (cudaMemsetAsync(scratch, 0, 2 * sizeof(uint32_t), st) != cudaSuccess) return WF_ERR_CUDA;
     return wf::launch_attn(mq, mk, mv, a, head_dim, grid, st) == cudaSuccess ? WF_OK : WF_ERR_CUDA;
 }
+
+// Test hook: every 32-bit word of the current device's scratch block set to
+// `word`, as a call whose bounded wait ran out leaves the status and timeout
+// site set (and a work counter past the units), so that a test can show the
+// next call starts clean.  Synchronous; not for use while a call runs.
+extern "C" int wf_noalloc_debug_fill_scratch(unsigned int word)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return WF_ERR_NO_DEVICE;
+    }
+    void *scratch = nullptr;
+    if (int s = scratch_for_current_device(dev, &scratch)) return s;
+    uint32_t fill[kNoAllocScratchBytes / sizeof(uint32_t)];
+    for (uint32_t &w : fill) w = word;
+    return cudaMemcpyToSymbol(g_noalloc_scratch, fill, sizeof(fill)) == cudaSuccess ? WF_OK
+                                                                                  : WF_ERR_CUDA;
+}

@@ -395,6 +395,15 @@ WF_API int wf_chunk_causal_attn_noalloc(int chunk_tokens, int n_wave_chunks, int
                                         const void *q_out, const void *k_cache,
                                         const void *v_cache, void *o, float *lse, void *stream);
 
+/* Test hook of the entry point above: sets every 32-bit word of the current
+ * device's scratch block to `word` (synchronously), the state a call whose
+ * bounded wait ran out leaves behind (status and timeout site set, the work
+ * counter past the last unit), so that a test can check that the next call
+ * starts clean.  It copies into the library's own block and allocates
+ * nothing.  Must not run while a call is in flight.  WF_OK, WF_ERR_NO_DEVICE,
+ * WF_ERR_CUDA. */
+WF_API int wf_noalloc_debug_fill_scratch(unsigned int word);
+
 #ifdef __cplusplus
 }
 #endif

@@ -10,7 +10,9 @@ scratch the first one left behind) its output must
   boundaries plus random rows) within the attention bar, and lse within 1e-3;
 - match wf_plan + wf_chunk_causal_attn on every row within the same bar;
 and every call after the first must leave the device's free memory and
-PyTorch's allocator statistics unchanged.
+PyTorch's allocator statistics unchanged.  A call after the scratch block was
+left dirty (every word set, through the library's test hook, as a timed-out
+call leaves status, timeout site and work counter) must still match the oracle.
 
 This file is named to be collected last, so a run that stops at the first
 failure has already run every other test; it also passes on its own.
@@ -115,6 +117,35 @@ def test_noalloc_matches_oracle_and_plan_api_twice(wf, L, W, Hh, H, D, r):
         lse_got = lse.cpu().numpy()[heads, rows]
         assert float(np.abs(lse_got - lse_orc).max()) <= 1e-3
         assert_attention_close(got.reshape(-1, D), ref, what + " vs plan API")
+
+
+def test_noalloc_after_a_dirty_scratch_block(wf):
+    """A call after one that left the scratch block dirty (status and timeout
+    site set, the work counter past the last unit: what a timed-out call
+    leaves) clears what must start at zero and matches the oracle."""
+    lib = wf.load()
+    L, W, Hh, H, D, r = 300, 4, 2, 3, 128, 5
+    q, kc, vc = _inputs(L, W, Hh, H, D, seed=99)
+    T = W * L
+    rows_s = sample_rows(L, W, n_random=24, seed=5)
+    rows = np.repeat(rows_s, H)
+    heads = np.tile(np.arange(H), rows_s.size)
+    cache = _oracle_cache(kc, vc, r, W, Hh)
+    o_orc, lse_orc = oracle.round_attention(cache, r, W, Hh, wi.bits(q.cpu()), rows, heads)
+    stream = torch.cuda.current_stream().cuda_stream
+    for word in (0xFFFFFFFF, 0x7FFFFFFF, 1):
+        torch.cuda.synchronize()
+        assert lib.wf_noalloc_debug_fill_scratch(word) == wf.WF_OK
+        o = torch.full_like(q, float("nan"))
+        lse = torch.full((H, T), float("nan"), dtype=torch.float32, device=q.device)
+        rc = lib.wf_chunk_causal_attn_noalloc(L, W, Hh, H, D, r, q.data_ptr(), kc.data_ptr(),
+                                              vc.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                              stream)
+        assert rc == wf.WF_OK, wf.status_string(rc)
+        got = o.cpu().float().numpy().reshape(T, H, D)
+        assert np.isfinite(got).all(), "fill %#x: rows left unwritten" % word
+        assert_attention_close(got[rows, heads], o_orc, "after fill %#x vs oracle" % word)
+        assert float(np.abs(lse.cpu().numpy()[heads, rows] - lse_orc).max()) <= 1e-3
 
 
 def test_noalloc_rejects_what_the_plan_rejects(wf):
