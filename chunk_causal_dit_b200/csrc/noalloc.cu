@@ -17,9 +17,8 @@
 // site, work counter) on its stream before the kernel runs, so calls whose work
 // overlaps on the GPU (different streams, no ordering between them) race on it
 // and must not be issued.  The kernel's timeout status is recorded in the block
-// but this entry point has no way to return it, so a call whose bounded wait
-// ran out (output partly written) cannot be told from a good one here: use the
-// plan API and wf_sync_status when the status is needed.
+// and wf_noalloc_sync_status reads it back (the call itself returns before the
+// kernel has run, so it cannot).
 #include <cudaTypedefs.h>
 
 #include <climits>
@@ -27,6 +26,7 @@
 #include <mutex>
 
 #include "wf.h"
+#include "wf_check.cuh"
 #include "wf_internal.h"
 
 namespace wf {
@@ -212,4 +212,31 @@ extern "C" int wf_noalloc_debug_fill_scratch(unsigned int word)
     for (uint32_t &w : fill) w = word;
     return cudaMemcpyToSymbol(g_noalloc_scratch, fill, sizeof(fill)) == cudaSuccess ? WF_OK
                                                                                   : WF_ERR_CUDA;
+}
+
+// The status the kernel recorded in the current device's scratch block, after
+// `stream` has finished: WF_ERR_TIMEOUT when a bounded wait ran out (output
+// partly written), WF_ERR_BOUNDS when a bounds check of the checked build
+// failed, else WF_OK.  Reads two words into host memory; clears nothing (the
+// next call does).  The block is shared by every call on the device, so the
+// answer covers the calls since the last one started.
+extern "C" int wf_noalloc_sync_status(void *stream)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return WF_ERR_NO_DEVICE;
+    }
+    void *scratch = nullptr;
+    if (int s = scratch_for_current_device(dev, &scratch)) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t words[2] = {0u, 0u};
+    if (cudaStreamSynchronize(st) != cudaSuccess ||
+        cudaMemcpyAsync(words, scratch, sizeof(words), cudaMemcpyDeviceToHost, st) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return WF_ERR_CUDA;
+    if (words[0] & wf::kStatusTimeout) return WF_ERR_TIMEOUT;
+    if (words[0] & wf::kStatusBounds) return WF_ERR_BOUNDS;
+    return WF_OK;
 }

@@ -59,6 +59,7 @@ SIGNATURES = {
     "wf_status_string": (ctypes.c_char_p, [_I]),
     "wf_chunk_causal_attn_noalloc": (_I, [_I, _I, _I, _I, _I, _L, _P, _P, _P, _P, _P, _P]),
     "wf_noalloc_debug_fill_scratch": (_I, [ctypes.c_uint]),
+    "wf_noalloc_sync_status": (_I, [_P]),
     "wf_quantize_q_fp8": (_I, [_P, _P, _P, _P, _P]),
     "wf_qk_norm_rope_append_fp8q": (_I, [_P, _L, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                          _P]),

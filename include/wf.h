@@ -385,9 +385,9 @@ WF_API const char *wf_status_string(int status);
  * looks up that block's device address (cudaGetSymbolAddress); make that first
  * call before any stream capture.  All calls on a device share the block: each
  * clears what must start at zero on its own stream, and calls that overlap on
- * the GPU race on it.  A device-side timeout is recorded in the block but not
- * reported here: such a call still returns WF_OK with o partly written, so a
- * caller that needs the status must use the plan API and wf_sync_status.  Returns WF_OK, WF_ERR_INVALID_ARG / WF_ERR_UNSUPPORTED for shapes or
+ * the GPU race on it.  A device-side timeout is recorded in the block; the
+ * call itself returns before the kernel runs (WF_OK, o then partly written),
+ * and wf_noalloc_sync_status below reads the recorded status back.  Returns WF_OK, WF_ERR_INVALID_ARG / WF_ERR_UNSUPPORTED for shapes or
  * pointers the plan API would reject, WF_ERR_NO_DEVICE, WF_ERR_DEVICE or
  * WF_ERR_CUDA. */
 WF_API int wf_chunk_causal_attn_noalloc(int chunk_tokens, int n_wave_chunks, int n_hist_chunks,
@@ -403,6 +403,15 @@ WF_API int wf_chunk_causal_attn_noalloc(int chunk_tokens, int n_wave_chunks, int
  * nothing.  Must not run while a call is in flight.  WF_OK, WF_ERR_NO_DEVICE,
  * WF_ERR_CUDA. */
 WF_API int wf_noalloc_debug_fill_scratch(unsigned int word);
+
+/* Wait for `stream`, then read the status the attention kernel recorded in the
+ * current device's scratch block: WF_ERR_TIMEOUT (a bounded device wait ran
+ * out; that call's o is partly written), WF_ERR_BOUNDS (a bounds check of the
+ * checked build failed), else WF_OK.  Copies two words to host memory and
+ * allocates nothing; clears nothing (the next call does).  The block is shared
+ * by every call on the device, so the answer covers the calls since the last
+ * one started.  WF_ERR_NO_DEVICE / WF_ERR_CUDA on a device error. */
+WF_API int wf_noalloc_sync_status(void *stream);
 
 #ifdef __cplusplus
 }

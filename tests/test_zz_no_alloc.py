@@ -146,6 +146,30 @@ def test_noalloc_after_a_dirty_scratch_block(wf):
         assert np.isfinite(got).all(), "fill %#x: rows left unwritten" % word
         assert_attention_close(got[rows, heads], o_orc, "after fill %#x vs oracle" % word)
         assert float(np.abs(lse.cpu().numpy()[heads, rows] - lse_orc).max()) <= 1e-3
+        assert lib.wf_noalloc_sync_status(stream) == wf.WF_OK
+
+
+def test_noalloc_status_query(wf):
+    """wf_noalloc_sync_status maps the block's status word the way wf_sync_status
+    maps a plan's: the timeout bit to WF_ERR_TIMEOUT, the bounds bit to
+    WF_ERR_BOUNDS (the words are planted through the test hook; no kernel is
+    made to time out), and a call that ran clean to WF_OK."""
+    lib = wf.load()
+    stream = torch.cuda.current_stream().cuda_stream
+    torch.cuda.synchronize()
+    for word, want in ((1, wf.WF_ERR_TIMEOUT), (2, wf.WF_ERR_BOUNDS), (3, wf.WF_ERR_TIMEOUT),
+                       (0, wf.WF_OK)):
+        assert lib.wf_noalloc_debug_fill_scratch(word) == wf.WF_OK
+        assert lib.wf_noalloc_sync_status(stream) == want, word
+    # a call clears the status left behind
+    assert lib.wf_noalloc_debug_fill_scratch(1) == wf.WF_OK
+    L, W, Hh, H, D, r = 200, 3, 1, 2, 64, 7
+    q, kc, vc = _inputs(L, W, Hh, H, D, seed=3)
+    o = torch.empty_like(q)
+    rc = lib.wf_chunk_causal_attn_noalloc(L, W, Hh, H, D, r, q.data_ptr(), kc.data_ptr(),
+                                          vc.data_ptr(), o.data_ptr(), None, stream)
+    assert rc == wf.WF_OK
+    assert lib.wf_noalloc_sync_status(stream) == wf.WF_OK
 
 
 def test_noalloc_rejects_what_the_plan_rejects(wf):
