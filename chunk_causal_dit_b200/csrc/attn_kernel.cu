@@ -21,9 +21,13 @@
 //   warps 0-3   softmax for query tile 0 (TMEM lanes 0..127, one row per thread)
 //   warps 4-7   softmax for query tile 1
 //   warp  8     scheduler + TMA producer: Q tiles, then K_j, V_j into a smem ring
-//   warp  9     MMA issuer (whole warp, one elected lane issues): S_x = Q_x K_j^T,
-//               O_x += P_x V_j
-//   warps 10-11 idle (they only give their registers to the softmax warpgroups)
+//   warps 9, 10 MMA issuers of query tiles 0 and 1 (whole warps, one elected
+//               lane issues): S_x = Q_x K_j^T, O_x += P_x V_j.  They take turns
+//               through a token, so the tensor pipe receives one fixed order
+//               (QK_0 QK_1 | PV_0 QK_0 | PV_1 QK_1 | ...); two issuers on two SMSPs
+//               instead of one halve the MMA-issue load that each SMSP's softmax
+//               warps share
+//   warp  11    idle (it only gives its registers to the softmax warpgroups)
 // Registers: launched at 168 per thread; the control warpgroup drops to 104 and
 // the two softmax warpgroups rise to 200 (setmaxnreg), which is exactly the
 // launch pool and leaves both paths spill-free.  The host refuses to launch if the compiled kernel does not use
@@ -91,18 +95,21 @@ struct Cfg {
     static constexpr uint32_t kS0 = 0, kS1 = 128, kO0 = 256, kO1 = 256 + D;
 };
 
+constexpr int kIssuers = 2;    // MMA issuers: warp kMmaWarp for query tile 0, the next for tile 1
+
 // Barrier indices inside the barrier block (8 bytes each).
 template <int S>
 struct Bars {
     static constexpr int q_full = 0, q_empty = 1, s_full = 2, p_ready = 4, o_final = 6,
                          drain = 8, sched_full = 9, sched_empty = 11, p_half = 13, kv_full = 15,
-                         kv_empty = 15 + S, count = 15 + 2 * S;
+                         kv_empty = 15 + S, turn = 15 + 2 * S, count = 17 + 2 * S;
 };
 
 // Wait-site codes recorded in DeviceWords::timeout_where.
 enum : uint32_t {
     kWhereProducerQ = 1, kWhereProducerKV = 2, kWhereMmaQ = 3, kWhereMmaKV = 4,
     kWhereMmaP = 5, kWhereSoftS = 6, kWhereSoftO = 7, kWhereDrain = 8, kWhereSched = 9,
+    kWhereMmaTurn = 10,
 };
 
 struct Ctl {
@@ -269,19 +276,20 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
 
     if (threadIdx.x == 0) {
         mbar_init(bar(B::q_full), 1);
-        mbar_init(bar(B::q_empty), 1);
+        mbar_init(bar(B::q_empty), kIssuers);
         for (int x = 0; x < 2; ++x) {
             mbar_init(bar(B::s_full + x), 1);
             mbar_init(bar(B::p_ready + x), 128);
             mbar_init(bar(B::p_half + x), 128);
             mbar_init(bar(B::o_final + x), 1);
             mbar_init(bar(B::sched_full + x), 1);
-            mbar_init(bar(B::sched_empty + x), 1 + kSoftmaxWarpsArrive);
+            mbar_init(bar(B::sched_empty + x), kIssuers + kSoftmaxWarpsArrive);
+            mbar_init(bar(B::turn + x), 1);
         }
-        mbar_init(bar(B::drain), 1);
+        mbar_init(bar(B::drain), kIssuers);
         for (int s = 0; s < S; ++s) {
             mbar_init(bar(B::kv_full + s), 1);
-            mbar_init(bar(B::kv_empty + s), 1);
+            mbar_init(bar(B::kv_empty + s), kIssuers);
         }
         *abort_flag = 0u;
         fence_barrier_init();
@@ -369,32 +377,54 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     if (f) wait_bar(bar(B::kv_full + s), (f - 1) & 1u, ctl, kWhereDrain, true);
                 }
             }
-        } else if (warp == kMmaWarp) {
-            // ---------------- MMA issuer ----------------
+        } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
+            // ---------------- MMA issuer of query tile x ----------------
             // The whole warp runs the loop and its waits (so the loop's values are
             // warp-uniform), and one elected lane issues every MMA, commit and
             // arrival.  Timed on B200 this issues ~15% more MMAs per cycle than a
             // single divergent lane, whose operands must be moved into uniform
             // registers one MMA at a time.
+            // The issuers of the two query tiles take turns: issuer x waits on
+            // turn + x and hands over by arriving on turn + (x ^ 1), so the
+            // tensor pipe receives one fixed order, QK_0(0) QK_1(0) | PV_0(j)
+            // QK_0(j+1) | PV_1(j) QK_1(j+1) | ...  Both wait for every K/V stage
+            // and unit, and both commit every stage release (the stage and
+            // q_empty barriers count two arrivals); an issuer whose tile lies
+            // past the chunk's end still takes its turns.  With each issuer on
+            // its own SMSP, the softmax warps that share an SMSP with one see
+            // half the MMA-issue traffic (clock64 stamps: the last P arrival of
+            // a tile 40-80 cycles earlier).
+            const int x = warp - kMmaWarp;
             const bool leader = elect_one_sync();
-            uint32_t stage = 0, kv_phase = 0, q_phase = 0;
-            uint32_t p_phase[2] = {0u, 0u};   // shared by p_half and p_ready (same cadence)
-            const uint32_t tS[2] = {tmem + C::kS0, tmem + C::kS1};
-            const uint32_t tO[2] = {tmem + C::kO0, tmem + C::kO1};
-            const uint32_t sQ[2] = {sq, sq + C::kQKTileBytes};
+            uint32_t stage = 0, kv_phase = 0, q_phase = 0, p_phase = 0, turn_phase = 0;
+            const uint32_t tSx = tmem + (x ? C::kS1 : C::kS0);
+            const uint32_t tOx = tmem + (x ? C::kO1 : C::kO0);
+            const uint32_t sQx = sq + x * C::kQKTileBytes;
             bool ok = true;
-            // bounded wait of the whole warp; false (in every lane) on timeout or abort
+            bool first_turn = x == 0;
             auto wait_all = [&](uint32_t b, uint32_t parity, uint32_t where) -> bool {
                 const bool r = wait_bar(b, parity, ctl, where);
                 return __all_sync(0xFFFFFFFFu, r);
             };
-            // take the next K/V stage in ring order, waiting until its copy landed
             auto next_stage = [&](uint32_t &st) -> bool {
                 st = stage;
                 const bool r = wait_all(bar(B::kv_full + stage), kv_phase, kWhereMmaKV);
                 if (++stage == static_cast<uint32_t>(S)) { stage = 0; kv_phase ^= 1u; }
                 tc_fence_after();
                 return r;
+            };
+            auto take_turn = [&]() -> bool {
+                if (first_turn) { first_turn = false; return true; }
+                const bool r = wait_all(bar(B::turn + x), turn_phase, kWhereMmaTurn);
+                turn_phase ^= 1u;
+                tc_fence_after();
+                return r;
+            };
+            auto pass_turn = [&]() {
+                tc_fence_before();
+                __syncwarp();
+                if (leader) mbar_arrive(bar(B::turn + (x ^ 1)));
+                __syncwarp();
             };
             for (uint32_t it = 0; ok; ++it) {
                 const uint32_t sl = it & 1u, ph = (it >> 1) & 1u;
@@ -404,76 +434,57 @@ chunk_causal_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 if (leader) mbar_arrive(bar(B::sched_empty + sl));
                 if (u >= p.n_units) break;
                 const Unit un = decode_unit(p, u);
+                const bool mine = x == 0 || un.has1;
                 if (!(ok = wait_all(bar(B::q_full), q_phase, kWhereMmaQ))) break;
                 q_phase ^= 1u;
                 uint32_t kst;
                 if (!(ok = next_stage(kst))) break;
+                if (!(ok = take_turn())) break;
                 if (leader) {
-                    issue_qk<D, F8>(tS[0], sQ[0], skv + kst * C::kTileBytes);
-                    umma_commit(bar(B::s_full + 0));
-                    if (un.has1) {
-                        issue_qk<D, F8>(tS[1], sQ[1], skv + kst * C::kTileBytes);
-                        umma_commit(bar(B::s_full + 1));
+                    if (mine) {
+                        issue_qk<D, F8>(tSx, sQx, skv + kst * C::kTileBytes);
+                        umma_commit(bar(B::s_full + x));
                     }
                     umma_commit(bar(B::kv_empty + kst));
                     if (un.n_kt == 1) umma_commit(bar(B::q_empty));
                 }
-                __syncwarp();
+                pass_turn();
                 for (int j = 0; ok && j < un.n_kt; ++j) {
                     const bool more = j + 1 < un.n_kt;
                     uint32_t vst, kst2 = 0;
                     if (!(ok = next_stage(vst))) break;
-                    // query tile 0: PV over the first 64 keys as soon as that half of P landed
-                    if (!(ok = wait_all(bar(B::p_half + 0), p_phase[0], kWhereMmaP))) break;
-                    tc_fence_after();
-                    if (leader) issue_pv_half<D>(tO[0], tS[0], skv + vst * C::kTileBytes, 0, j > 0);
-                    __syncwarp();
-                    if (!(ok = wait_all(bar(B::p_ready + 0), p_phase[0], kWhereMmaP))) break;
-                    p_phase[0] ^= 1u;
-                    tc_fence_after();
-                    if (leader) issue_pv_half<D>(tO[0], tS[0], skv + vst * C::kTileBytes, 1, true);
-                    __syncwarp();
-                    if (more) {
-                        if (!(ok = next_stage(kst2))) break;
-                        if (leader) {
-                            issue_qk<D, F8>(tS[0], sQ[0], skv + kst2 * C::kTileBytes);
-                            umma_commit(bar(B::s_full + 0));
-                        }
-                    } else if (leader) {
-                        umma_commit(bar(B::o_final + 0));
-                    }
-                    __syncwarp();
-                    // query tile 1
-                    if (un.has1) {
-                        if (!(ok = wait_all(bar(B::p_half + 1), p_phase[1], kWhereMmaP))) break;
+                    if (more && !(ok = next_stage(kst2))) break;
+                    if (!(ok = take_turn())) break;
+                    if (mine) {
+                        if (!(ok = wait_all(bar(B::p_half + x), p_phase, kWhereMmaP))) break;
                         tc_fence_after();
-                        if (leader)
-                            issue_pv_half<D>(tO[1], tS[1], skv + vst * C::kTileBytes, 0, j > 0);
+                        if (leader) issue_pv_half<D>(tOx, tSx, skv + vst * C::kTileBytes, 0, j > 0);
                         __syncwarp();
-                        if (!(ok = wait_all(bar(B::p_ready + 1), p_phase[1], kWhereMmaP))) break;
-                        p_phase[1] ^= 1u;
+                        if (!(ok = wait_all(bar(B::p_ready + x), p_phase, kWhereMmaP))) break;
+                        p_phase ^= 1u;
                         tc_fence_after();
-                        if (leader)
-                            issue_pv_half<D>(tO[1], tS[1], skv + vst * C::kTileBytes, 1, true);
+                        if (leader) issue_pv_half<D>(tOx, tSx, skv + vst * C::kTileBytes, 1, true);
                         __syncwarp();
                     }
                     if (leader) {
+                        if (more) {
+                            if (mine) {
+                                issue_qk<D, F8>(tSx, sQx, skv + kst2 * C::kTileBytes);
+                                umma_commit(bar(B::s_full + x));
+                            }
+                        } else if (mine) {
+                            umma_commit(bar(B::o_final + x));
+                        }
                         umma_commit(bar(B::kv_empty + vst));
                         if (more) {
-                            if (un.has1) {
-                                issue_qk<D, F8>(tS[1], sQ[1], skv + kst2 * C::kTileBytes);
-                                umma_commit(bar(B::s_full + 1));
-                            }
                             umma_commit(bar(B::kv_empty + kst2));
                             if (j + 2 == un.n_kt) umma_commit(bar(B::q_empty));
-                        } else if (un.has1) {
-                            umma_commit(bar(B::o_final + 1));
                         }
                     }
-                    __syncwarp();
+                    pass_turn();
                 }
             }
-            // every MMA issued by the leader completes before TMEM is released
+            // every MMA issued by this warp's leader completes before TMEM is released
             if (leader) umma_commit(bar(B::drain));
             __syncwarp();
             wait_bar(bar(B::drain), 0u, ctl, kWhereDrain, true);
