@@ -72,11 +72,14 @@ static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl == kThreads * kRegsLau
               "the register re-split must add up to the launch pool");
 constexpr int kSoftmaxWarpsArrive = 8;      // sched_empty: one arrival per softmax warp
 // Pair e of a 32-pair block takes the FMA-pipe exp2 when e % kEmulatePeriod ==
-// kEmulatePeriod - 1; 0 keeps every exponential on MUFU.  Timed on B200, sending
-// 12.5%, 25% or 33% of the exponentials to the FMA pipe made the kernel slower
-// (during its exp phase a tile's softmax is one warp per SMSP, which the extra
-// instructions lengthen more than MUFU relief shortens), so the default is 0.
-constexpr int kEmulatePeriod = 0;
+// kEmulatePeriod - 1 (period 3: 10 of every 32 pairs); 0 keeps every
+// exponential on MUFU.  Timed on B200: with a single MMA-issuing warp, sending
+// 12.5-33% of the exponentials to the FMA pipe made the kernel slower (the
+// MMA-side chain set the period); with one issuer per query tile, period 3 or 4
+// is 0.6-1.5% faster than MUFU alone, period 8 no faster, period 2 14% slower.
+// Period 3 keeps every instantiation spill-free (period 4 spills 16 bytes).
+// The polynomial's relative error (7.5e-5) is far below P's bf16 rounding.
+constexpr int kEmulatePeriod = 3;
 
 // F8: Q and K arrive as E4M3 codes (one byte per element, one 128-byte
 // swizzle atom per row at D = 128) with fp32 scales; V, P and O stay as in the
