@@ -360,6 +360,7 @@ def run_ours(args, rank, world, local):
     h2d_gbs = 3 * tensor_bytes / (min(h2d_ms) * 1e-3) / 1e9
 
     clk = clocks.summary(t_wall0, t_wall1)
+    head_block = plan.head_block(r0, fp8)      # the attention's unit order (steady state)
     block = None
     if not args.no_block and w.H * w.D in wi.BLOCK_WIDTHS:
         del q, k, v, x, hq, hk_, hv_, ho, pipe
@@ -404,6 +405,7 @@ def run_ours(args, rank, world, local):
             "workload": w.name,
             "heads": w.H, "head_dim": w.D, "chunk_tokens": w.L, "wave_chunks": w.n_wave,
             "history_chunks": w.n_hist, "wave_tokens": w.T, "attention": args.attn,
+            "attn_unit_order": "heads in blocks of %d" % head_block,
             "parallelism": "replica%d (independent wave rounds, no data-path collective)" % world,
             "l2": l2_note((append_bytes + 2 * w.R * w.L * w.H * w.D * 2) / 1e6),
         },
