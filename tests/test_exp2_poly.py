@@ -5,7 +5,8 @@ gen_exp2_poly.py).  Here the kernel's float32 steps are replayed in numpy:
 j = round(x) via the 1.5*2^23 shift, f = x - j, Horner in float32, scale by 2^j;
 the result is compared with exp2 in float64 over x in [-126, 8], the range the
 softmax feeds it (scores minus a running maximum that is at most 2^8 stale).
-The kernel's default keeps every exponential on MUFU; this checks the optional path.
+The attention kernel sends a third of the exponential pairs through this path
+(the rest through MUFU ex2.approx); this checks its error bound.
 """
 import os
 import re
