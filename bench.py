@@ -148,6 +148,15 @@ class ClockSampler:
                 return
             self._stop.wait(self.interval)
 
+    def wait_ready(self, n=3, timeout_s=2.0):
+        """Wait (at most timeout_s) until the sampler has taken n samples, so that a
+        slow first NVML query on a fresh process cannot leave a short timed region
+        without any sample."""
+        t_end = time.time() + timeout_s
+        while self._thread is not None and len(self.samples) < n and self.error is None \
+                and time.time() < t_end:
+            time.sleep(0.002)
+
     def stop(self):
         if self._thread is not None:
             self._stop.set()
@@ -280,7 +289,7 @@ def run_ours(args, rank, world, local):
           for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
-    time.sleep(0.02)
+    clocks.wait_ready()
     barrier(dist, dev)
     torch.cuda.synchronize(dev)
     t_wall0 = time.time()
@@ -539,7 +548,7 @@ def measure_single_layer(w, steps, warmup, dev, peaks, fp8=False, seed=0):
     torch.cuda.synchronize(dev)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
     clocks = ClockSampler(dev.index)
-    time.sleep(0.02)
+    clocks.wait_ready()
     torch.cuda.synchronize(dev)
     t0 = time.time()
     for i in range(steps):
@@ -632,7 +641,7 @@ def measure_round_loop(w, rounds, warmup, dev, peaks, seed=0, dist=None):
     aev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             for _ in range(w.layers)] for _ in range(rounds)]
     clocks = ClockSampler(dev.index)
-    time.sleep(0.02)
+    clocks.wait_ready()
     barrier(dist, dev)
     torch.cuda.synchronize(dev)
     t0 = time.time()
@@ -726,7 +735,7 @@ def measure_vae_stage(steps, warmup, dev, peaks, seed=0):
     torch.cuda.synchronize(dev)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
     clocks = ClockSampler(dev.index)
-    time.sleep(0.02)
+    clocks.wait_ready()
     torch.cuda.synchronize(dev)
     t0 = time.time()
     for i in range(steps):
@@ -1179,7 +1188,7 @@ def run_block_round_loop(args, rank, world, local):
     rev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(rounds)]
     clocks = ClockSampler(local)
-    time.sleep(0.02)
+    clocks.wait_ready()
     barrier(dist, dev)
     torch.cuda.synchronize(dev)
     t_wall0 = time.time()
